@@ -1,0 +1,200 @@
+"""Context-parallel attention on one B200: Python binding of ``libcp_attn.so``.
+
+This module only marshals arguments: every step of the computation runs in the
+CUDA library built from ``csrc/`` (see ``include/cp_attn.h`` for the C ABI). It
+uses PyTorch for device memory and streams. There is no CPU fallback: importing
+raises when the library is missing, and every call raises on a non-zero status.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcp_attn.so")
+
+CONTIGUOUS, ZIGZAG, ULYSSES = 0, 1, 2
+LAYOUTS = {"contiguous": CONTIGUOUS, "zigzag": ZIGZAG, "ulysses": ULYSSES}
+
+STATUS = {0: "CP_OK", -1: "CP_ERR_INVALID_ARG", -2: "CP_ERR_UNSUPPORTED", -3: "CP_ERR_ALIGNMENT",
+          -4: "CP_ERR_CUDA", -5: "CP_ERR_TIMEOUT", -6: "CP_ERR_WORKSPACE"}
+
+# Every function the header declares, with its ctypes signature.
+_P, _I, _I64, _SZ, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+SIGNATURES = {
+    "cp_attn_plan": (_I, [ctypes.POINTER(_P), _I, _I, _I, _I, _I, _I, _I, _F]),
+    "cp_attn_plan_destroy": (_I, [_P]),
+    "cp_attn_plan_tile_counts": (_I64, [_P, _P]),
+    "cp_attn_plan_num_items": (_I64, [_P]),
+    "cp_attn_workspace_bytes": (_SZ, [_P, _I]),
+    "cp_attn_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
+    "cp_attn_fwd_partials": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
+    "cp_merge_partials": (_I, [_I, _I64, _I, _P, _P, _P, _P, _P]),
+    "cp_layout_permute": (_I, [_P, _I, _P, _P, _I, _P]),
+    "cp_layout_index_map_len": (_I64, [_P]),
+    "cp_layout_index_map": (_I, [_P, _P, _P]),
+    "cp_attn_check": (_I, [_P, _P]),
+    "cp_status_string": (ctypes.c_char_p, [_I]),
+    "cp_debug_wait_timeout_probe": (_I, [_P, _I, _P]),
+}
+
+
+class CpAttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({lib().cp_status_string(status).decode()})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m context_long_sequence_cp_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise CpAttnError(fn, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+class Plan:
+    """A context-parallel attention plan (wraps ``cp_attn_plan``)."""
+
+    def __init__(self, B: int, H: int, S: int, D: int, N: int, causal: bool, layout: str = "zigzag",
+                 softmax_scale: float = 0.0):
+        self.B, self.H, self.S, self.D, self.N = B, H, S, D, N
+        self.causal, self.layout = bool(causal), layout
+        self.scale = softmax_scale if softmax_scale > 0 else 1.0 / math.sqrt(D)
+        h = ctypes.c_void_p()
+        _check("cp_attn_plan", lib().cp_attn_plan(ctypes.byref(h), B, H, S, D, N, int(bool(causal)),
+                                                   LAYOUTS[layout], float(softmax_scale)))
+        self._h = h
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib().cp_attn_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def tile_counts(self):
+        arr = (ctypes.c_int64 * self.N)()
+        tot = lib().cp_attn_plan_tile_counts(self._h, ctypes.cast(arr, ctypes.c_void_p))
+        if tot < 0:
+            raise CpAttnError("cp_attn_plan_tile_counts", int(tot))
+        return list(arr), int(tot)
+
+    def num_items(self) -> int:
+        return int(lib().cp_attn_plan_num_items(self._h))
+
+    def workspace_bytes(self, with_partials: bool = False) -> int:
+        return int(lib().cp_attn_workspace_bytes(self._h, int(with_partials)))
+
+    def index_map_len(self) -> int:
+        return int(lib().cp_layout_index_map_len(self._h))
+
+    @property
+    def rows(self) -> int:
+        return self.B * self.S * self.H
+
+
+def attn_fwd(plan: Plan, q, k, v, o=None, lse=None, workspace=None, stream=None):
+    """Fused forward (``cp_attn_fwd``): returns (o, lse)."""
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(plan.B, plan.H, plan.S, dtype=torch.float32, device=q.device)
+    nws = plan.workspace_bytes(False)
+    if workspace is None and nws > 0:
+        workspace = torch.empty(nws, dtype=torch.uint8, device=q.device)
+    _check("cp_attn_fwd", lib().cp_attn_fwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                            _ptr(workspace), _stream(stream)))
+    return o, lse
+
+
+def attn_fwd_partials(plan: Plan, q, k, v, o_parts=None, lse_parts=None, stream=None):
+    """Per-ring-step partials (``cp_attn_fwd_partials``): ([N, rows, D] fp32, [N, rows] fp32)."""
+    if o_parts is None:
+        o_parts = torch.empty(plan.N, plan.rows, plan.D, dtype=torch.float32, device=q.device)
+    if lse_parts is None:
+        lse_parts = torch.empty(plan.N, plan.rows, dtype=torch.float32, device=q.device)
+    _check("cp_attn_fwd_partials", lib().cp_attn_fwd_partials(plan.handle, _ptr(q), _ptr(k), _ptr(v),
+                                                              _ptr(o_parts), _ptr(lse_parts), None,
+                                                              _stream(stream)))
+    return o_parts, lse_parts
+
+
+def merge_partials(o_parts, lse_parts, o_out=None, lse_out=None, stream=None):
+    """Merge [P, rows, D] fp32 partials (``cp_merge_partials``): (bf16 [rows, D], fp32 [rows])."""
+    P, rows, D = o_parts.shape
+    if o_out is None:
+        o_out = torch.empty(rows, D, dtype=torch.bfloat16, device=o_parts.device)
+    if lse_out is None:
+        lse_out = torch.empty(rows, dtype=torch.float32, device=o_parts.device)
+    _check("cp_merge_partials", lib().cp_merge_partials(P, rows, D, _ptr(o_parts), _ptr(lse_parts),
+                                                        _ptr(o_out), _ptr(lse_out), _stream(stream)))
+    return o_out, lse_out
+
+
+def layout_permute(plan: Plan, x, direction: int, out=None, stream=None):
+    """Index-mapped layout copy (``cp_layout_permute``); bit-exact."""
+    if out is None:
+        out = torch.empty_like(x)
+    _check("cp_layout_permute", lib().cp_layout_permute(plan.handle, int(direction), _ptr(x), _ptr(out),
+                                                        x.element_size(), _stream(stream)))
+    return out
+
+
+def layout_index_map(plan: Plan, device="cuda", stream=None):
+    """The layout's int64 index map (``cp_layout_index_map``)."""
+    out = torch.empty(plan.index_map_len(), dtype=torch.int64, device=device)
+    _check("cp_layout_index_map", lib().cp_layout_index_map(plan.handle, _ptr(out), _stream(stream)))
+    return out
+
+
+def check(plan: Plan, stream=None) -> int:
+    """``cp_attn_check``: synchronise and return the recorded status (0 = ok)."""
+    return int(lib().cp_attn_check(plan.handle, _stream(stream)))
+
+
+def debug_wait_timeout_probe(plan: Plan, timeout_us: int, stream=None):
+    _check("cp_debug_wait_timeout_probe",
+           lib().cp_debug_wait_timeout_probe(plan.handle, int(timeout_us), _stream(stream)))
+
+
+def status_string(status: int) -> str:
+    return lib().cp_status_string(int(status)).decode()

@@ -1,0 +1,379 @@
+// api.cu — the C ABI (include/cp_attn.h): plan construction, argument
+// validation, TMA descriptor encoding and kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "attn_fwd.h"
+#include "cp_attn.h"
+#include "geometry.h"
+
+using namespace cpattn;
+
+struct cp_attn_plan_s {
+  int B, H, S, D, N, causal, layout;
+  float scale;
+  Geometry g;                       // attention view of the kernel
+  int lse_B, lse_H;
+  int64_t lse_S;
+  std::vector<WorkItem> items;      // sorted work list
+  std::vector<int64_t> tile_counts; // executed tile pairs per virtual rank
+  WorkItem* d_items = nullptr;      // device copy of the work list
+  int* d_status = nullptr;          // device status word
+  int device = -1;
+};
+
+namespace {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per in-kernel wait
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 4-D view (D, Hh, T, NR*B) of a bf16 tensor stored [NR*B][T][Hh][D]; box of
+// 64 x 1 x 128 x 1 elements (128 B x 128 rows) with the 128-byte swizzle.
+int encode_view(CUtensorMap* map, const void* base, const Geometry& g, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return CP_ERR_CUDA;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(g.Hh),
+                              static_cast<cuuint64_t>(g.T), static_cast<cuuint64_t>(g.NR) * g.B};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(g.Hh) * D * 2,
+                                 static_cast<cuuint64_t>(g.T) * g.Hh * D * 2};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kTile), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CP_OK : CP_ERR_CUDA;
+}
+
+// Executed key tiles of a work item (both query tiles) over ring steps [t0, t1).
+void item_cost(const Geometry& g, int rq, int qp, int t0, int t1, int* c0n, int* c1n) {
+  KeyTileWalk w;
+  w.init(g, rq, qp * kPair, t0, t1);
+  int rk, kt, c0, c1;
+  *c0n = *c1n = 0;
+  while (w.next(rk, kt, c0, c1)) {
+    *c0n += c0 != kSkip;
+    *c1n += c1 != kSkip;
+  }
+}
+
+int ensure_device(cp_attn_plan_s* p) {
+  if (p->d_items != nullptr) return CP_OK;
+  return CP_ERR_CUDA;
+}
+
+int launch_view(cp_attn_plan_s* p, const Geometry& g, const void* q, const void* k, const void* v, void* o,
+                float* lse, float* o_part, float* lse_part, int t0, int t1, bool partial, cudaStream_t st) {
+  FwdLaunch L;
+  std::memset(&L, 0, sizeof(L));
+  int rc;
+  if ((rc = encode_view(&L.tm_q, q, g, p->D)) != CP_OK) return rc;
+  if ((rc = encode_view(&L.tm_k, k, g, p->D)) != CP_OK) return rc;
+  if ((rc = encode_view(&L.tm_v, v, g, p->D)) != CP_OK) return rc;
+  FwdParams& P = L.params;
+  P.g = g;
+  P.t_begin = t0;
+  P.t_end = t1;
+  P.scale_log2 = p->scale * 1.4426950408889634f;
+  P.items = p->d_items;
+  P.n_items = static_cast<int>(p->items.size());
+  P.o = static_cast<__nv_bfloat16*>(o);
+  P.lse = lse;
+  P.lse_B = p->lse_B;
+  P.lse_H = p->lse_H;
+  P.lse_S = p->lse_S;
+  P.o_part = o_part;
+  P.lse_part = lse_part;
+  P.status = p->d_status;
+  P.wait_limit_ns = kWaitLimitNs;
+  return launch_attn_fwd(L, p->D, partial, st) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+PermuteArgs permute_args(const cp_attn_plan_s* p, int direction, int elem_bytes) {
+  PermuteArgs a;
+  a.kind = p->layout == CP_LAYOUT_ULYSSES ? 1 : 0;
+  a.direction = direction;
+  a.N = p->N;
+  a.B = p->B;
+  a.S = p->S;
+  a.H = p->H;
+  a.D = p->D;
+  a.zigzag = p->layout == CP_LAYOUT_ZIGZAG;
+  a.elem_bytes = elem_bytes;
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int cp_attn_plan(cp_attn_plan_t* out, int B, int H, int S, int D, int N, int causal, int layout,
+                 float softmax_scale) {
+  if (out == nullptr) return CP_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (B <= 0 || H <= 0 || S <= 0 || N <= 0) return CP_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return CP_ERR_INVALID_ARG;
+  if (layout < CP_LAYOUT_CONTIGUOUS || layout > CP_LAYOUT_ULYSSES) return CP_ERR_INVALID_ARG;
+  if (!(softmax_scale <= 0.f || std::isfinite(softmax_scale))) return CP_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return CP_ERR_UNSUPPORTED;
+  if (S % N != 0) return CP_ERR_UNSUPPORTED;
+  if (layout == CP_LAYOUT_ZIGZAG && S % (2 * N) != 0) return CP_ERR_UNSUPPORTED;
+  if (layout == CP_LAYOUT_ULYSSES && (H % N != 0 || causal)) return CP_ERR_UNSUPPORTED;
+  // int32 indexing limits of the kernels: tokens per view, view row blocks, TMA dims.
+  if (static_cast<int64_t>(B) * N > (1 << 20) || static_cast<int64_t>(B) * S * H * D > (int64_t(1) << 40))
+    return CP_ERR_UNSUPPORTED;
+
+  cp_attn_plan_s* p = new (std::nothrow) cp_attn_plan_s();
+  if (p == nullptr) return CP_ERR_INVALID_ARG;
+  p->B = B;
+  p->H = H;
+  p->S = S;
+  p->D = D;
+  p->N = N;
+  p->causal = causal;
+  p->layout = layout;
+  p->scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p->lse_B = B;
+  p->lse_H = H;
+  p->lse_S = S;
+  Geometry& g = p->g;
+  if (layout == CP_LAYOUT_ULYSSES) {
+    g = Geometry{1, N * B, H / N, S, S, 0, 0};
+  } else {
+    g = Geometry{N, B, H, S / N, layout == CP_LAYOUT_ZIGZAG ? S / (2 * N) : S / N, layout == CP_LAYOUT_ZIGZAG,
+                 causal};
+  }
+
+  // Work list: every (rank, batch, head, query-tile pair) with its executed key tiles.
+  const int npairs = (g.T + kPair - 1) / kPair;
+  p->tile_counts.assign(N, 0);
+  p->items.reserve(static_cast<size_t>(g.NR) * g.B * g.Hh * npairs);
+  for (int r = 0; r < g.NR; ++r) {
+    for (int b = 0; b < g.B; ++b) {
+      for (int qp = 0; qp < npairs; ++qp) {
+        int c0, c1;
+        item_cost(g, r, qp, 0, g.NR, &c0, &c1);   // same for every head
+        for (int h = 0; h < g.Hh; ++h) {
+          p->items.push_back(WorkItem{r * g.B + b, h, qp, c0 + c1});
+          const int rank = layout == CP_LAYOUT_ULYSSES ? b / B : r;
+          p->tile_counts[rank] += c0 + c1;
+        }
+      }
+    }
+  }
+  // Items that read the same keys/values (same batch and head) are kept together
+  // so that the ones running at the same time share them in L2; within a group
+  // the most expensive come first.
+  std::stable_sort(p->items.begin(), p->items.end(), [&](const WorkItem& a, const WorkItem& b) {
+    const int ba = a.rb % g.B, bb = b.rb % g.B;
+    if (ba != bb) return ba < bb;
+    if (a.h != b.h) return a.h < b.h;
+    return a.cost > b.cost;
+  });
+
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0) {
+    cudaGetDevice(&p->device);
+    const size_t bytes = p->items.size() * sizeof(WorkItem);
+    bool ok = cudaMalloc(&p->d_items, bytes > 0 ? bytes : sizeof(WorkItem)) == cudaSuccess &&
+              cudaMalloc(&p->d_status, sizeof(int)) == cudaSuccess &&
+              cudaMemcpy(p->d_items, p->items.data(), bytes, cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMemset(p->d_status, 0, sizeof(int)) == cudaSuccess;
+    if (!ok) {
+      cudaFree(p->d_items);
+      cudaFree(p->d_status);
+      p->d_items = nullptr;
+      p->d_status = nullptr;
+    }
+  } else {
+    cudaGetLastError();   // clear the "no device" error
+  }
+  *out = p;
+  return CP_OK;
+}
+
+int cp_attn_plan_destroy(cp_attn_plan_t plan) {
+  if (plan == nullptr) return CP_OK;
+  if (plan->d_items != nullptr) cudaFree(plan->d_items);
+  if (plan->d_status != nullptr) cudaFree(plan->d_status);
+  delete plan;
+  return CP_OK;
+}
+
+int64_t cp_attn_plan_tile_counts(cp_attn_plan_t plan, int64_t* per_rank) {
+  if (plan == nullptr) return CP_ERR_INVALID_ARG;
+  int64_t tot = 0;
+  for (int r = 0; r < plan->N; ++r) {
+    if (per_rank != nullptr) per_rank[r] = plan->tile_counts[r];
+    tot += plan->tile_counts[r];
+  }
+  return tot;
+}
+
+int64_t cp_attn_plan_num_items(cp_attn_plan_t plan) {
+  if (plan == nullptr) return CP_ERR_INVALID_ARG;
+  return static_cast<int64_t>(plan->items.size());
+}
+
+size_t cp_attn_workspace_bytes(cp_attn_plan_t plan, int with_partials) {
+  if (plan == nullptr) return 0;
+  if (plan->layout == CP_LAYOUT_ULYSSES && !with_partials)
+    return 4 * static_cast<size_t>(plan->B) * plan->S * plan->H * plan->D * 2;
+  return 0;
+}
+
+int cp_attn_fwd(cp_attn_plan_t plan, const void* q, const void* k, const void* v, void* o, float* lse,
+                void* workspace, cp_stream_t stream) {
+  if (plan == nullptr || q == nullptr || k == nullptr || v == nullptr || o == nullptr) return CP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(workspace))
+    return CP_ERR_ALIGNMENT;
+  int rc = ensure_device(plan);
+  if (rc != CP_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (plan->layout != CP_LAYOUT_ULYSSES)
+    return launch_view(plan, plan->g, q, k, v, o, lse, nullptr, nullptr, 0, plan->g.NR, false, st);
+
+  if (workspace == nullptr) return CP_ERR_WORKSPACE;
+  const size_t tensor = static_cast<size_t>(plan->B) * plan->S * plan->H * plan->D * 2;
+  char* ws = static_cast<char*>(workspace);
+  void* gq = ws;
+  void* gk = ws + tensor;
+  void* gv = ws + 2 * tensor;
+  void* go = ws + 3 * tensor;
+  const PermuteArgs fwd = permute_args(plan, 0, 2);
+  if (launch_permute(fwd, q, gq, st) != cudaSuccess || launch_permute(fwd, k, gk, st) != cudaSuccess ||
+      launch_permute(fwd, v, gv, st) != cudaSuccess)
+    return CP_ERR_CUDA;
+  rc = launch_view(plan, plan->g, gq, gk, gv, go, lse, nullptr, nullptr, 0, 1, false, st);
+  if (rc != CP_OK) return rc;
+  return launch_permute(permute_args(plan, 1, 2), go, o, st) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+int cp_attn_fwd_partials(cp_attn_plan_t plan, const void* q, const void* k, const void* v, float* o_parts,
+                         float* lse_parts, void* workspace, cp_stream_t stream) {
+  (void)workspace;
+  if (plan == nullptr || q == nullptr || k == nullptr || v == nullptr || o_parts == nullptr ||
+      lse_parts == nullptr)
+    return CP_ERR_INVALID_ARG;
+  if (plan->layout == CP_LAYOUT_ULYSSES) return CP_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_parts) || !aligned16(lse_parts))
+    return CP_ERR_ALIGNMENT;
+  int rc = ensure_device(plan);
+  if (rc != CP_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t rows = static_cast<int64_t>(plan->B) * plan->S * plan->H;
+  for (int t = 0; t < plan->N; ++t) {
+    rc = launch_view(plan, plan->g, q, k, v, nullptr, nullptr, o_parts + t * rows * plan->D, lse_parts + t * rows,
+                     t, t + 1, true, st);
+    if (rc != CP_OK) return rc;
+  }
+  return CP_OK;
+}
+
+int cp_merge_partials(int num_parts, int64_t rows, int D, const float* o_parts, const float* lse_parts,
+                      void* o_out, float* lse_out, cp_stream_t stream) {
+  if (num_parts < 1 || num_parts > 64 || rows < 0) return CP_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return CP_ERR_UNSUPPORTED;
+  if (rows > 0 && (o_parts == nullptr || lse_parts == nullptr || o_out == nullptr)) return CP_ERR_INVALID_ARG;
+  if (!aligned16(o_parts) || !aligned16(o_out) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse_out) & 3u))
+    return CP_ERR_ALIGNMENT;
+  return launch_merge(num_parts, rows, D, o_parts, lse_parts, static_cast<__nv_bfloat16*>(o_out), lse_out,
+                      static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? CP_OK
+             : CP_ERR_CUDA;
+}
+
+int cp_layout_permute(cp_attn_plan_t plan, int direction, const void* in, void* out, int elem_bytes,
+                      cp_stream_t stream) {
+  if (plan == nullptr || in == nullptr || out == nullptr) return CP_ERR_INVALID_ARG;
+  if (direction != 0 && direction != 1) return CP_ERR_INVALID_ARG;
+  if (elem_bytes != 2 && elem_bytes != 4) return CP_ERR_INVALID_ARG;
+  if (!aligned16(in) || !aligned16(out)) return CP_ERR_ALIGNMENT;
+  const PermuteArgs a = permute_args(plan, direction, elem_bytes);
+  const int64_t unit_elems =
+      a.kind == 0 ? static_cast<int64_t>(plan->H) * plan->D : static_cast<int64_t>(plan->H / plan->N) * plan->D;
+  if ((unit_elems * elem_bytes) % 16 != 0) return CP_ERR_UNSUPPORTED;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) return CP_ERR_CUDA;
+  return launch_permute(a, in, out, static_cast<cudaStream_t>(stream)) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+int64_t cp_layout_index_map_len(cp_attn_plan_t plan) {
+  if (plan == nullptr) return CP_ERR_INVALID_ARG;
+  return plan->layout == CP_LAYOUT_ULYSSES ? static_cast<int64_t>(plan->N) * plan->B * plan->S
+                                           : static_cast<int64_t>(plan->B) * plan->S;
+}
+
+int cp_layout_index_map(cp_attn_plan_t plan, int64_t* map_out, cp_stream_t stream) {
+  if (plan == nullptr || map_out == nullptr) return CP_ERR_INVALID_ARG;
+  if (!aligned16(map_out)) return CP_ERR_ALIGNMENT;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) return CP_ERR_CUDA;
+  return launch_index_map(permute_args(plan, 0, 2), map_out, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? CP_OK
+             : CP_ERR_CUDA;
+}
+
+int cp_attn_check(cp_attn_plan_t plan, cp_stream_t stream) {
+  if (plan == nullptr) return CP_ERR_INVALID_ARG;
+  if (plan->d_status == nullptr) return CP_ERR_CUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return CP_ERR_CUDA;
+  int status = 0;
+  if (cudaMemcpy(&status, plan->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return CP_ERR_CUDA;
+  if (status != 0) {
+    cudaMemset(plan->d_status, 0, sizeof(int));
+    return status;
+  }
+  return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+const char* cp_status_string(int status) {
+  switch (status) {
+    case CP_OK: return "ok";
+    case CP_ERR_INVALID_ARG: return "invalid argument";
+    case CP_ERR_UNSUPPORTED: return "unsupported shape or layout";
+    case CP_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case CP_ERR_CUDA: return "CUDA error or no device";
+    case CP_ERR_TIMEOUT: return "in-kernel wait timed out";
+    case CP_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int cp_debug_wait_timeout_probe(cp_attn_plan_t plan, int timeout_us, cp_stream_t stream) {
+  if (plan == nullptr || timeout_us < 1 || timeout_us > 1000000) return CP_ERR_INVALID_ARG;
+  if (plan->d_status == nullptr) return CP_ERR_CUDA;
+  return launch_wait_probe(plan->d_status, static_cast<uint64_t>(timeout_us) * 1000ull,
+                           static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? CP_OK
+             : CP_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,507 @@
+// attn_fwd.cu — context-parallel attention forward on sm_100a (tcgen05 + TMEM + TMA).
+//
+// What it computes (page "序列与上下文并行", section "上下文并行：注意力本身切分"):
+// for every query tile of every virtual rank r, the key/value tiles of ranks
+// (r + t) mod N, t = 0..N-1, are visited in that ring order and folded into one
+// running online-softmax state (row max m, row sum l, unnormalised O), which is
+// the incremental merge of the per-step partials; at the end O/l and the
+// logsumexp m + log l are written. Scores are scaled by 1/sqrt(D) and masked
+// keys are -inf (page "Tensor并行与算子拆分", section "注意力的并行化优化"); the
+// causal mask uses global positions (section "工程实践" of the first page).
+// Key tiles wholly above the causal diagonal are never loaded or multiplied.
+// In partial mode the kernel visits a single ring step and writes that step's
+// normalised fp32 (O_t, lse_t) instead.
+//
+// Kernel design (one CTA per SM, persistent over a work list; 12 warps):
+//   warps 0-3  softmax warpgroup 0: query tile 0 of the item, one row per thread
+//   warps 4-7  softmax warpgroup 1: query tile 1 of the item
+//   warp  8    allocates TMEM; lane 0 issues every tcgen05.mma
+//   warp  9    lane 0 issues every TMA load
+//   warps 10-11 idle
+// TMEM (512 columns x 128 lanes): S0 [0,128) S1 [128,256) O0 [256,256+D)
+// O1 [256+D, 256+2D). P (bf16, packed 2 per column) overwrites the first 64
+// columns of its S tile and feeds the PV product straight from TMEM.
+// Shared memory: Q0, Q1 and a ring of NS key/value stages, each a 128 x D bf16
+// tile stored as D/64 column blocks of 128 rows x 128 B with the 128-byte swizzle
+// that TMA writes and the UMMA descriptors read.
+//
+// Per key tile j the MMA warp issues: PV0(j), S0(j+1), PV1(j), S1(j+1), so the
+// tensor core computes one query tile's products while the other warpgroup
+// runs its softmax. Rescaling of O is lazy: only when a row max grows by more
+// than 2^8 (in the exp2 domain) is O multiplied in TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+
+#include "attn_fwd.h"
+#include "geometry.h"
+#include "sm100.cuh"
+
+namespace cpattn {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kThreads = 384;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows by > 256x
+
+template <int D>
+struct Cfg {
+  static constexpr int kTileBytes = kTile * D * 2;               // one 128 x D bf16 tile
+  static constexpr int kBlocks = D / 64;                         // 128-byte column blocks
+  static constexpr int kBlockBytes = kTile * 128;                // 16 KB
+  static constexpr int kStages = D == 128 ? 4 : 6;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kOCol = 256;
+  static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);   // Q K^T, both K-major
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);    // P V, V is MN-major
+};
+
+template <int D>
+struct alignas(1024) Smem {
+  __nv_bfloat16 q[2][kTile * D];
+  __nv_bfloat16 kv[Cfg<D>::kStages][kTile * D];
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[Cfg<D>::kStages];
+  uint64_t kv_empty[Cfg<D>::kStages];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
+
+template <int D>
+__device__ __forceinline__ void issue_s(uint32_t tS, uint32_t q_addr, uint32_t k_addr) {
+  // S = Q K^T over K = D in steps of 16: four steps per 128-byte column block.
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * Cfg<D>::kBlockBytes + (kk & 3) * 32;
+    const uint64_t a = smem_desc_sw128(q_addr + off, 16, 1024);
+    const uint64_t b = smem_desc_sw128(k_addr + off, 16, 1024);
+    umma_ss(tS, a, b, Cfg<D>::kIdescS, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint32_t v_addr, bool accumulate) {
+  // O (+)= P V over K = 128 keys in steps of 16: P from TMEM (8 packed columns per
+  // step), V from shared memory as an MN-major operand (8-key groups 1024 B apart,
+  // 64-column blocks kBlockBytes apart).
+#pragma unroll
+  for (int kk = 0; kk < kTile / 16; ++kk) {
+    const uint64_t b = smem_desc_sw128(v_addr + kk * 2048, Cfg<D>::kBlockBytes, 1024);
+    umma_ts(tO, tP + kk * 8, b, Cfg<D>::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+}  // namespace
+
+template <int D, bool PARTIAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  Smem<D>& sm = *reinterpret_cast<Smem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = lane_id();
+  const Geometry g = p.g;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&sm.q_full), 1);
+    mbar_init(smem_addr(&sm.q_empty), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(smem_addr(&sm.kv_full[s]), 1);
+      mbar_init(smem_addr(&sm.kv_empty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_addr(&sm.s_full[i]), 1);
+      mbar_init(smem_addr(&sm.p_full[i]), 128);
+      mbar_init(smem_addr(&sm.o_done[i]), 1);
+    }
+    mbar_init(smem_addr(&sm.drain), 1);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_addr(&sm.tmem_base), C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 9 && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = sm.tmem_base;
+  WaitCtl ctl{&sm.abort, p.status, p.wait_limit_ns};
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_q = l2_policy_evict_first();
+      const uint64_t pol_kv = l2_policy_evict_last();
+      int q_iter = 0;
+      int kv_idx = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
+        const WorkItem w = p.items[it];
+        const int rq = w.rb / g.B;
+        const int bv = w.rb - rq * g.B;
+        const int q0 = w.qp * kPair;
+        if (q_iter > 0) ok = mbar_wait(smem_addr(&sm.q_empty), (q_iter - 1) & 1, ctl);
+        if (!ok) break;
+        const uint32_t qbar = smem_addr(&sm.q_full);
+        mbar_arrive_expect_tx(qbar, 2 * C::kTileBytes);
+        for (int i = 0; i < 2; ++i)
+          for (int blk = 0; blk < C::kBlocks; ++blk)
+            tma_load_4d(smem_addr(&sm.q[i][0]) + blk * C::kBlockBytes, &tm_q, qbar, blk * 64, w.h,
+                        q0 + i * kTile, w.rb, pol_q);
+        ++q_iter;
+        KeyTileWalk walk;
+        walk.init(g, rq, q0, p.t_begin, p.t_end);
+        int rk, kt, c0, c1;
+        while (ok && walk.next(rk, kt, c0, c1)) {
+          const int rbk = rk * g.B + bv;
+          for (int which = 0; which < 2; ++which) {
+            const int stage = kv_idx % C::kStages;
+            const int round = kv_idx / C::kStages;
+            if (round > 0) ok = mbar_wait(smem_addr(&sm.kv_empty[stage]), (round - 1) & 1, ctl);
+            if (!ok) break;
+            const uint32_t bar = smem_addr(&sm.kv_full[stage]);
+            mbar_arrive_expect_tx(bar, C::kTileBytes);
+            const CUtensorMap* map = which == 0 ? &tm_k : &tm_v;
+            for (int blk = 0; blk < C::kBlocks; ++blk)
+              tma_load_4d(smem_addr(&sm.kv[stage][0]) + blk * C::kBlockBytes, map, bar, blk * 64,
+                          w.h, kt * kTile, rbk, pol_kv);
+            ++kv_idx;
+          }
+        }
+      }
+      if (!ok) {
+        // Abort: let every load this thread issued land before the CTA exits.
+        const uint64_t lim = p.wait_limit_ns;
+        for (int idx = kv_idx - C::kStages; idx < kv_idx; ++idx)
+          if (idx >= 0)
+            mbar_wait_drain(smem_addr(&sm.kv_full[idx % C::kStages]), (idx / C::kStages) & 1, lim);
+        if (q_iter > 0) mbar_wait_drain(smem_addr(&sm.q_full), (q_iter - 1) & 1, lim);
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t tS0 = tbase, tS1 = tbase + 128;
+      const uint32_t tO0 = tbase + C::kOCol, tO1 = tbase + C::kOCol + D;
+      const uint32_t q_addr0 = smem_addr(&sm.q[0][0]), q_addr1 = smem_addr(&sm.q[1][0]);
+      int q_iter = 0, kv_idx = 0;
+      int p_cnt0 = 0, p_cnt1 = 0;
+      bool ok = true, issued = false;
+      for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
+        const WorkItem w = p.items[it];
+        const int rq = w.rb / g.B;
+        const int q0 = w.qp * kPair;
+        // Count the PV products of each query tile so the last one can signal o_done.
+        int n_pv0 = 0, n_pv1 = 0;
+        {
+          KeyTileWalk cnt;
+          cnt.init(g, rq, q0, p.t_begin, p.t_end);
+          int rk, kt, c0, c1;
+          while (cnt.next(rk, kt, c0, c1)) {
+            n_pv0 += c0 != kSkip;
+            n_pv1 += c1 != kSkip;
+          }
+        }
+        ok = mbar_wait(smem_addr(&sm.q_full), q_iter & 1, ctl);
+        if (!ok) break;
+        ++q_iter;
+        tc_fence_after();
+        KeyTileWalk walk;
+        walk.init(g, rq, q0, p.t_begin, p.t_end);
+        int rk, kt, cur0, cur1;
+        if (!walk.next(rk, kt, cur0, cur1)) {
+          umma_commit(smem_addr(&sm.q_empty));
+          continue;
+        }
+        // First key tile: both S products.
+        int kst = kv_idx % C::kStages;
+        ok = mbar_wait(smem_addr(&sm.kv_full[kst]), (kv_idx / C::kStages) & 1, ctl);
+        if (!ok) break;
+        ++kv_idx;
+        tc_fence_after();
+        const uint32_t k_addr0 = smem_addr(&sm.kv[kst][0]);
+        if (cur0 != kSkip) {
+          issue_s<D>(tS0, q_addr0, k_addr0);
+          umma_commit(smem_addr(&sm.s_full[0]));
+        }
+        if (cur1 != kSkip) {
+          issue_s<D>(tS1, q_addr1, k_addr0);
+          umma_commit(smem_addr(&sm.s_full[1]));
+        }
+        issued = true;
+        umma_commit(smem_addr(&sm.kv_empty[kst]));
+        int seen0 = 0, seen1 = 0;
+        for (;;) {
+          int nrk, nkt, nxt0, nxt1;
+          const bool has_next = walk.next(nrk, nkt, nxt0, nxt1);
+          const int vst = kv_idx % C::kStages;
+          ok = mbar_wait(smem_addr(&sm.kv_full[vst]), (kv_idx / C::kStages) & 1, ctl);
+          if (!ok) break;
+          ++kv_idx;
+          tc_fence_after();
+          const uint32_t v_addr = smem_addr(&sm.kv[vst][0]);
+          int nst = 0;
+          uint32_t nk_addr = 0;
+          // Query tile 0: PV0(cur), then S0(next).
+          if (cur0 != kSkip) {
+            ok = mbar_wait(smem_addr(&sm.p_full[0]), p_cnt0 & 1, ctl);
+            if (!ok) break;
+            ++p_cnt0;
+            tc_fence_after();
+            issue_pv<D>(tO0, tS0, v_addr, seen0 > 0);
+            if (++seen0 == n_pv0) umma_commit(smem_addr(&sm.o_done[0]));
+          }
+          if (has_next) {
+            nst = kv_idx % C::kStages;
+            ok = mbar_wait(smem_addr(&sm.kv_full[nst]), (kv_idx / C::kStages) & 1, ctl);
+            if (!ok) break;
+            ++kv_idx;
+            tc_fence_after();
+            nk_addr = smem_addr(&sm.kv[nst][0]);
+            if (nxt0 != kSkip) {
+              issue_s<D>(tS0, q_addr0, nk_addr);
+              umma_commit(smem_addr(&sm.s_full[0]));
+            }
+          }
+          // Query tile 1: PV1(cur), then S1(next).
+          if (cur1 != kSkip) {
+            ok = mbar_wait(smem_addr(&sm.p_full[1]), p_cnt1 & 1, ctl);
+            if (!ok) break;
+            ++p_cnt1;
+            tc_fence_after();
+            issue_pv<D>(tO1, tS1, v_addr, seen1 > 0);
+            if (++seen1 == n_pv1) umma_commit(smem_addr(&sm.o_done[1]));
+          }
+          if (has_next && nxt1 != kSkip) {
+            issue_s<D>(tS1, q_addr1, nk_addr);
+            umma_commit(smem_addr(&sm.s_full[1]));
+          }
+          if (!ok) break;
+          if (has_next) umma_commit(smem_addr(&sm.kv_empty[nst]));
+          umma_commit(smem_addr(&sm.kv_empty[vst]));
+          if (!has_next) break;
+          cur0 = nxt0;
+          cur1 = nxt1;
+        }
+        if (!ok) break;
+        umma_commit(smem_addr(&sm.q_empty));
+      }
+      if (issued) {
+        // Every tensor-core op (and the arrivals of its commits) must finish before
+        // TMEM is freed and the CTA exits; on the abort path too.
+        umma_commit(smem_addr(&sm.drain));
+        mbar_wait_drain(smem_addr(&sm.drain), 0, p.wait_limit_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = warp >> 2;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tS = tbase + lane_off + wg * 128;
+    const uint32_t tO = tbase + lane_off + C::kOCol + wg * D;
+    const float sl2 = p.scale_log2;
+    int s_cnt = 0, od_cnt = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
+      const WorkItem w = p.items[it];
+      const int rq = w.rb / g.B;
+      const int bv = w.rb - rq * g.B;
+      const int q_first = w.qp * kPair;
+      const int tl = q_first + wg * kTile + row;
+      const bool valid = tl < g.T;
+      const int64_t gq = global_pos(g, rq, valid ? tl : g.T - 1);
+      float m_run = -INFINITY, l_run = 0.f;
+      int ntile = 0;
+      KeyTileWalk walk;
+      walk.init(g, rq, q_first, p.t_begin, p.t_end);
+      int rk, kt, c0, c1;
+      while (walk.next(rk, kt, c0, c1)) {
+        const int cls = wg == 0 ? c0 : c1;
+        if (cls == kSkip) continue;
+        ok = mbar_wait(smem_addr(&sm.s_full[wg]), s_cnt & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++s_cnt;
+        tc_fence_after();
+        float s[kTile];
+        tmem_ld128(tS, reinterpret_cast<uint32_t*>(s));
+        if (cls == kMasked) {
+          const int lim = valid ? column_limit(g, rk, kt * kTile, gq) : 0;
+#pragma unroll
+          for (int j = 0; j < kTile; ++j) s[j] = j < lim ? s[j] : -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int j = 1; j < kTile; ++j) mx = fmaxf(mx, s[j]);
+        const float m_tile = mx * sl2;
+        const float m_new = fmaxf(m_run, m_tile);
+        const bool resc = m_new - m_run > kRescaleThreshold;   // false while both are -inf
+        float alpha = 1.f;
+        if (resc) {
+          alpha = ex2_approx(m_run - m_new);   // 0 when m_run = -inf
+          m_run = m_new;
+          l_run *= alpha;
+        }
+        const float m_use = m_run == -INFINITY ? 0.f : m_run;
+        float lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float e0 = ex2_approx(fmaf(s[c * 32 + 2 * j], sl2, -m_use));
+            const float e1 = ex2_approx(fmaf(s[c * 32 + 2 * j + 1], sl2, -m_use));
+            lsum += e0 + e1;
+            pk[j] = pack_bf16x2(e0, e1);
+          }
+          tmem_st16(tS + c * 16, pk);
+        }
+        if (ntile > 0 && __any_sync(0xffffffffu, resc)) {
+          // O holds the previous PV products (complete: this tile's s_full was
+          // committed after them) and the next PV waits for p_full: rescale in place.
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c, o);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            tmem_st32(tO + c, o);
+          }
+        }
+        l_run += lsum;
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(smem_addr(&sm.p_full[wg]));
+        ++ntile;
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      const int64_t row_id = (static_cast<int64_t>(w.rb) * g.T + tl) * g.Hh + w.h;
+      if (ntile > 0) {
+        ok = mbar_wait(smem_addr(&sm.o_done[wg]), od_cnt & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++od_cnt;
+        tc_fence_after();
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c, o);
+          if (valid) {
+            if (PARTIAL) {
+              float4* dst = reinterpret_cast<float4*>(p.o_part + row_id * D + c);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                dst[j] = make_float4(__uint_as_float(o[4 * j]) * inv, __uint_as_float(o[4 * j + 1]) * inv,
+                                     __uint_as_float(o[4 * j + 2]) * inv,
+                                     __uint_as_float(o[4 * j + 3]) * inv);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(p.o + row_id * D + c);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                uint4 v;
+                v.x = pack_bf16x2(__uint_as_float(o[8 * j + 0]) * inv, __uint_as_float(o[8 * j + 1]) * inv);
+                v.y = pack_bf16x2(__uint_as_float(o[8 * j + 2]) * inv, __uint_as_float(o[8 * j + 3]) * inv);
+                v.z = pack_bf16x2(__uint_as_float(o[8 * j + 4]) * inv, __uint_as_float(o[8 * j + 5]) * inv);
+                v.w = pack_bf16x2(__uint_as_float(o[8 * j + 6]) * inv, __uint_as_float(o[8 * j + 7]) * inv);
+                dst[j] = v;
+              }
+            }
+          }
+        }
+        if (valid) {
+          const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+          if (PARTIAL) {
+            p.lse_part[row_id] = lse;
+          } else if (p.lse != nullptr) {
+            const int64_t li = (static_cast<int64_t>(bv % p.lse_B) * p.lse_H + (bv / p.lse_B) * g.Hh + w.h) *
+                                   p.lse_S + gq;
+            p.lse[li] = lse;
+          }
+        }
+      } else if (valid) {
+        // No allowed key at all in the visited steps: O = 0, lse = -inf.
+        if (PARTIAL) {
+          float4* dst = reinterpret_cast<float4*>(p.o_part + row_id * D);
+          for (int j = 0; j < D / 4; ++j) dst[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          p.lse_part[row_id] = -INFINITY;
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(p.o + row_id * D);
+          for (int j = 0; j < D / 8; ++j) dst[j] = make_uint4(0, 0, 0, 0);
+          if (p.lse != nullptr) {
+            const int64_t li = (static_cast<int64_t>(bv % p.lse_B) * p.lse_H + (bv / p.lse_B) * g.Hh + w.h) *
+                                   p.lse_S + gq;
+            p.lse[li] = -INFINITY;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------- host side
+
+namespace {
+
+template <int D, bool PARTIAL>
+cudaError_t launch_impl(const FwdLaunch& L, cudaStream_t stream) {
+  const size_t smem = sizeof(Smem<D>) + 1024;
+  auto kern = attn_fwd_kernel<D, PARTIAL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int grid = L.params.n_items < sms ? L.params.n_items : sms;
+  if (grid <= 0) return cudaSuccess;
+  kern<<<grid, kThreads, smem, stream>>>(L.tm_q, L.tm_k, L.tm_v, L.params);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd(const FwdLaunch& L, int D, bool partial, cudaStream_t stream) {
+  if (D == 128) return partial ? launch_impl<128, true>(L, stream) : launch_impl<128, false>(L, stream);
+  if (D == 64) return partial ? launch_impl<64, true>(L, stream) : launch_impl<64, false>(L, stream);
+  return cudaErrorInvalidValue;
+}
+
+size_t attn_fwd_smem_bytes(int D) {
+  return D == 128 ? sizeof(Smem<128>) + 1024 : sizeof(Smem<64>) + 1024;
+}
+
+}  // namespace cpattn

@@ -1,0 +1,57 @@
+// attn_fwd.h — launch parameters of the attention forward kernel (internal).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "geometry.h"
+
+namespace cpattn {
+
+struct FwdParams {
+  Geometry g;
+  int t_begin, t_end;          // ring steps visited: [t_begin, t_end)
+  float scale_log2;            // softmax scale * log2(e)
+  const WorkItem* items;       // device work list
+  int n_items;
+  __nv_bfloat16* o;            // fused output, view layout [NR*B][T][Hh][D]
+  float* lse;                  // natural [lse_B][lse_H][lse_S]; may be null
+  int lse_B, lse_H;
+  int64_t lse_S;
+  float* o_part;               // partial mode: [rows][D], row = (rb*T + tl)*Hh + h
+  float* lse_part;             // partial mode: [rows]
+  int* status;                 // device status word (0 = ok)
+  uint64_t wait_limit_ns;      // budget of one in-kernel wait
+};
+
+struct FwdLaunch {
+  CUtensorMap tm_q, tm_k, tm_v;   // 4-D views (D, Hh, T, NR*B) of q, k, v
+  FwdParams params;
+};
+
+cudaError_t launch_attn_fwd(const FwdLaunch& L, int D, bool partial, cudaStream_t stream);
+size_t attn_fwd_smem_bytes(int D);
+
+// merge.cu
+cudaError_t launch_merge(int num_parts, int64_t rows, int D, const float* o_parts,
+                         const float* lse_parts, __nv_bfloat16* o_out, float* lse_out,
+                         cudaStream_t stream);
+
+// permute.cu
+struct PermuteArgs {
+  int kind;          // 0: contiguous/zigzag token rows; 1: Ulysses head-group runs
+  int direction;     // 0: forward gather, 1: inverse
+  int N, B, S, H, D;
+  int zigzag;
+  int elem_bytes;
+};
+cudaError_t launch_permute(const PermuteArgs& a, const void* in, void* out, cudaStream_t stream);
+cudaError_t launch_index_map(const PermuteArgs& a, int64_t* map_out, cudaStream_t stream);
+
+// probe.cu
+cudaError_t launch_wait_probe(int* status, uint64_t limit_ns, cudaStream_t stream);
+
+}  // namespace cpattn

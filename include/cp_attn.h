@@ -1,0 +1,224 @@
+/*
+ * cp_attn.h — C ABI of the B200 (sm_100a) context-parallel attention library.
+ *
+ * The method (page "序列与上下文并行", ai-infra-wiki, section
+ * "上下文并行：注意力本身切分"): the sequence of S tokens is split over N ranks;
+ * each rank holds its own Q/K/V block; K/V blocks travel around a ring so that
+ * at ring step t rank r computes its Q block against the K/V block of rank
+ * (r + t) mod N; the per-step partial results (O, logsumexp) are merged by
+ * online softmax, which yields exactly full softmax attention. For causal
+ * attention a zigzag assignment of chunks to ranks balances the work (same
+ * section). Here the N ranks are virtual: all of them run on one GPU as tile
+ * and CTA scheduling.
+ *
+ * Attention itself (page "Tensor并行与算子拆分", aiknowledge.cn, section
+ * "注意力的并行化优化"): O = softmax(Q K^T * scale + mask) V with masked
+ * scores set to -inf; scale defaults to 1/sqrt(D). The causal mask keeps key
+ * j for query i iff pos(j) <= pos(i) in GLOBAL token positions (page
+ * "序列与上下文并行", section "工程实践": positions are global under context
+ * parallelism).
+ *
+ * Layouts (element order, outermost first; all tensors dense, no padding):
+ *   natural              [B][S][H][D]
+ *   CP_LAYOUT_CONTIGUOUS [N][B][S/N][H][D]  rank r holds tokens [r*S/N, (r+1)*S/N)
+ *                        (page "序列并行：超长序列训练", guijiagi.com, split diagram)
+ *   CP_LAYOUT_ZIGZAG     [N][B][2C][H][D], C = S/(2N): rank r holds chunk r then
+ *                        chunk 2N-1-r of 2N equal chunks (the zigzag reading)
+ *   CP_LAYOUT_ULYSSES    inputs/outputs as sequence shards [N][B][S/N][H][D];
+ *                        internally head groups [N][B][S][H/N][D], group g holding
+ *                        heads [g*H/N, (g+1)*H/N) (page "序列并行：超长序列训练",
+ *                        UlyssesAttention example: all-to-all, local attention over
+ *                        the full sequence, all-to-all back)
+ *   lse                  float32 [B][H][S], natural token order, natural log of
+ *                        the sum of exp of the scaled scores.
+ *
+ * Conventions for every entry point:
+ *   - Status codes: CP_OK (0) or a negative CP_ERR_*; no exception crosses the ABI.
+ *   - Device pointers must be 16-byte aligned (CP_ERR_ALIGNMENT otherwise).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Entry points
+ *     that take a stream only enqueue work: they neither allocate device memory
+ *     nor synchronise, except cp_attn_check, which synchronises `stream`.
+ *   - The caller owns every input, output and workspace buffer. A plan owns only
+ *     its host schedule and a small device table (work list + status word)
+ *     allocated by cp_attn_plan and freed by cp_attn_plan_destroy.
+ *   - Plans are immutable after creation; concurrent calls on one plan with
+ *     distinct outputs and workspaces are safe.
+ *   - Kernel waits are bounded: a wait that runs out sets the plan's status word,
+ *     the kernel returns early, and the next cp_attn_check reports CP_ERR_TIMEOUT.
+ */
+#ifndef CP_ATTN_H_
+#define CP_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CP_API __attribute__((visibility("default")))
+#else
+#define CP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, passed as an opaque pointer so this header needs no CUDA header. */
+typedef void* cp_stream_t;
+
+enum {
+  CP_OK = 0,
+  CP_ERR_INVALID_ARG = -1,   /* null pointer, non-positive size, bad enum value */
+  CP_ERR_UNSUPPORTED = -2,   /* D not in {64,128}; S not divisible by N (2N for zigzag);
+                                H not divisible by N (Ulysses); sizes beyond int32 indexing */
+  CP_ERR_ALIGNMENT = -3,     /* a device pointer is not 16-byte aligned */
+  CP_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed, or no device */
+  CP_ERR_TIMEOUT = -5,       /* a bounded in-kernel wait ran out (reported by cp_attn_check) */
+  CP_ERR_WORKSPACE = -6      /* workspace pointer null or smaller than required */
+};
+
+typedef enum {
+  CP_LAYOUT_CONTIGUOUS = 0,
+  CP_LAYOUT_ZIGZAG = 1,
+  CP_LAYOUT_ULYSSES = 2
+} cp_layout_t;
+
+typedef struct cp_attn_plan_s* cp_attn_plan_t;
+
+/*
+ * Build a plan for B batches, H heads, S tokens, head dim D (64 or 128), N
+ * virtual ranks, causal (0/1), a layout, and a softmax scale (<= 0 selects
+ * 1/sqrt(D)). The plan holds the ring schedule (per rank r and step t the
+ * key/value rank (r+t) mod N; per (query tile, key tile) pair of 128 tokens
+ * the class full / masked / skipped), the work list of query-tile pairs sorted
+ * by descending executed-tile count, and, when a CUDA device is present, a
+ * device copy of the work list plus a status word. Without a device the plan
+ * is still created (host queries work) and every launch returns CP_ERR_CUDA.
+ * Ulysses plans take causal = 0 only (CP_ERR_UNSUPPORTED otherwise).
+ * On success *out receives the plan; on failure *out is set to NULL.
+ */
+CP_API int cp_attn_plan(cp_attn_plan_t* out, int B, int H, int S, int D, int N, int causal,
+                 int layout, float softmax_scale);
+
+/* Free a plan and its device table. NULL is accepted. Not to be called while a
+ * launch on the plan may still be running (synchronise first). */
+CP_API int cp_attn_plan_destroy(cp_attn_plan_t plan);
+
+/*
+ * Executed 128x128 (query tile, key tile) pairs of each virtual rank, summed
+ * over ring steps, batches and heads: per_rank[N] (host memory, may be NULL).
+ * Returns the total over ranks, or a negative status. For the zigzag causal
+ * layout every rank gets the same count; for the contiguous causal layout rank
+ * r's count grows with r (the load imbalance of the causal section).
+ */
+CP_API int64_t cp_attn_plan_tile_counts(cp_attn_plan_t plan, int64_t* per_rank);
+
+/* Number of work items (pairs of 128-row query tiles) in the plan's work list. */
+CP_API int64_t cp_attn_plan_num_items(cp_attn_plan_t plan);
+
+/*
+ * Workspace bytes needed by cp_attn_fwd (with_partials = 0) or
+ * cp_attn_fwd_partials (with_partials = 1). 0 for contiguous/zigzag fused
+ * calls; 4 * B*S*H*D*2 bytes (Q, K, V and O head groups) for Ulysses.
+ */
+CP_API size_t cp_attn_workspace_bytes(cp_attn_plan_t plan, int with_partials);
+
+/*
+ * Fused forward: O and lse of full softmax attention, computed by visiting for
+ * each query tile of each virtual rank r the key/value tiles of ranks
+ * (r+t) mod N for t = 0..N-1 in that order, merging every step into one
+ * running online-softmax state (the incremental merge of the context-parallel
+ * section), skipping key tiles that lie wholly above the causal diagonal.
+ *   q, k, v : bf16, in the plan's layout (see above), device
+ *   o       : bf16, same layout and size as q, device (written)
+ *   lse     : float32 [B][H][S] natural token order, device (written); may be NULL
+ *   workspace : device, cp_attn_workspace_bytes(plan, 0) bytes (NULL if 0)
+ * q, k, v must not overlap o or workspace.
+ */
+CP_API int cp_attn_fwd(cp_attn_plan_t plan, const void* q, const void* k, const void* v,
+                void* o, float* lse, void* workspace, cp_stream_t stream);
+
+/*
+ * Unfused forward (contiguous/zigzag only; CP_ERR_UNSUPPORTED for Ulysses):
+ * the per-ring-step partials of the context-parallel section, unmerged.
+ *   o_parts   : float32 [N][rows][D], device (written)
+ *   lse_parts : float32 [N][rows], device (written)
+ * with rows = N*B*(S/N)*H ordered like q's tokens and heads,
+ * row = ((r*B + b)*(S/N) + tl)*H + h, and part t holding rank r's rows
+ * against the key/value block of rank (r+t) mod N. A row with no allowed key in
+ * a step gets O = 0, lse = -inf. O_t is normalised (the softmax-weighted mean
+ * over that step's keys) and lse_t is natural-log. cp_merge_partials over the
+ * N parts gives O in q's layout and lse in row order.
+ */
+CP_API int cp_attn_fwd_partials(cp_attn_plan_t plan, const void* q, const void* k, const void* v,
+                         float* o_parts, float* lse_parts, void* workspace,
+                         cp_stream_t stream);
+
+/*
+ * Merge num_parts partials per row (same section: online-softmax merge):
+ *   M = max_t lse_t, lse = M + ln sum_t exp(lse_t - M), O = sum_t exp(lse_t - lse) O_t.
+ * Partials with lse_t = -inf contribute nothing; rows whose partials are all
+ * -inf give O = 0 and lse = -inf.
+ *   o_parts   : float32 [num_parts][rows][D], device
+ *   lse_parts : float32 [num_parts][rows], device
+ *   o_out     : bf16 [rows][D], device (written, round-to-nearest-even)
+ *   lse_out   : float32 [rows], device (written); may be NULL
+ * D must be 64 or 128; 1 <= num_parts <= 64.
+ */
+CP_API int cp_merge_partials(int num_parts, int64_t rows, int D, const float* o_parts,
+                      const float* lse_parts, void* o_out, float* lse_out,
+                      cp_stream_t stream);
+
+/*
+ * Layout permutation (the all-to-all of the pages done as an index-mapped copy
+ * on one GPU; page "4. 序列并行" (5688vip.com) simulates it the same way, by
+ * index mapping). Elements are opaque: elem_bytes is 2 or 4.
+ *   contiguous/zigzag: direction 0 = natural [B][S][H][D] -> rank-major,
+ *                      direction 1 = rank-major -> natural.
+ *   Ulysses:           direction 0 = shards [N][B][S/N][H][D] -> groups [N][B][S][H/N][D],
+ *                      direction 1 = groups -> shards.
+ * in/out: device, B*S*H*D*elem_bytes bytes each, must not overlap. Bit-exact copy.
+ */
+CP_API int cp_layout_permute(cp_attn_plan_t plan, int direction, const void* in, void* out,
+                      int elem_bytes, cp_stream_t stream);
+
+/* Length of the index map written by cp_layout_index_map: B*S for
+ * contiguous/zigzag (one entry per token), N*B*S for Ulysses (one entry per
+ * (group, batch, token) run of H/N heads). */
+CP_API int64_t cp_layout_index_map_len(cp_attn_plan_t plan);
+
+/*
+ * Write the layout's int64 index map (device, cp_layout_index_map_len entries):
+ *   contiguous/zigzag: map[(r*B + b)*(S/N) + tl] = natural flat token b*S + pos,
+ *                      pos = the global position of rank r's local token tl;
+ *   Ulysses: map[(g*B + b)*S + s] = ((rho*B + b)*(S/N) + s mod (S/N))*N + g,
+ *            rho = s div (S/N): the run of the shards tensor (viewed as runs of
+ *            H/N heads) that lands at group g, batch b, token s.
+ * Direction-0 permutation is out[i] = in[map[i]] over rows/runs.
+ */
+CP_API int cp_layout_index_map(cp_attn_plan_t plan, int64_t* map_out, cp_stream_t stream);
+
+/*
+ * Synchronise `stream`, then report the first error recorded since the last
+ * check: CP_ERR_TIMEOUT if a bounded in-kernel wait ran out (the status word is
+ * then cleared), CP_ERR_CUDA on an asynchronous CUDA error, else CP_OK.
+ */
+CP_API int cp_attn_check(cp_attn_plan_t plan, cp_stream_t stream);
+
+/* Static, human-readable text for a status code. */
+CP_API const char* cp_status_string(int status);
+
+/*
+ * Fault-detection self-test of the bounded wait used by every kernel: launches
+ * one CTA that waits on a shared-memory barrier that nothing ever arrives on,
+ * with a limit of timeout_us microseconds, then records the outcome in the
+ * plan's status word and returns. The host sees it through cp_attn_check
+ * (expected: CP_ERR_TIMEOUT). No fault, trap or unbounded spin is involved.
+ * 1 <= timeout_us <= 1000000.
+ */
+CP_API int cp_debug_wait_timeout_probe(cp_attn_plan_t plan, int timeout_us, cp_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CP_ATTN_H_ */

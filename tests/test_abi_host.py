@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI: no GPU needed, no compute calls.
+
+* the library builds, loads and exports every function ``include/cp_attn.h`` declares;
+* plan creation validates its arguments;
+* the plan's executed tile-pair counts equal the oracle's brute-force enumeration.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import context_long_sequence_cp_b200 as cp
+from context_long_sequence_cp_b200 import build as cpbuild
+from oracle import schedule as Sch
+from workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "cp_attn.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    cpbuild.build()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(cp_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("cp_attn_plan", "cp_attn_fwd", "cp_merge_partials", "cp_layout_permute",
+                     "cp_layout_index_map", "cp_attn_fwd_partials", "cp_attn_check"):
+        assert required in names
+    assert sorted(cp.SIGNATURES) == names
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", cp.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(\S+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(cp.lib(), name) is not None
+    # nothing else leaks out of the library's C++/CUDA internals
+    assert not [s for s in exported if s.startswith("_ZN6cpattn")]
+
+
+def test_status_strings():
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert cp.status_string(code) not in ("", "unknown status")
+    assert cp.status_string(-99) == "unknown status"
+
+
+def _plan_status(*args):
+    h = ctypes.c_void_p()
+    rc = cp.lib().cp_attn_plan(ctypes.byref(h), *args)
+    if rc == 0:
+        cp.lib().cp_attn_plan_destroy(h)
+    else:
+        assert h.value is None
+    return rc
+
+
+def test_plan_argument_validation():
+    Z, C, U = cp.ZIGZAG, cp.CONTIGUOUS, cp.ULYSSES
+    assert _plan_status(1, 2, 256, 64, 4, 0, C, 0.0) == 0
+    assert _plan_status(1, 2, 256, 96, 4, 0, C, 0.0) == -2          # D not 64/128
+    assert _plan_status(1, 2, 250, 64, 4, 0, C, 0.0) == -2          # S % N
+    assert _plan_status(1, 2, 255, 64, 5, 1, Z, 0.0) == -2          # S % 2N for zigzag
+    assert _plan_status(1, 6, 256, 64, 4, 0, U, 0.0) == -2          # H % N for Ulysses
+    assert _plan_status(1, 8, 256, 64, 4, 1, U, 0.0) == -2          # causal Ulysses
+    assert _plan_status(0, 2, 256, 64, 4, 0, C, 0.0) == -1          # B <= 0
+    assert _plan_status(1, 2, 256, 64, 0, 0, C, 0.0) == -1          # N <= 0
+    assert _plan_status(1, 2, 256, 64, 4, 2, C, 0.0) == -1          # causal not 0/1
+    assert _plan_status(1, 2, 256, 64, 4, 0, 7, 0.0) == -1          # bad layout
+    assert cp.lib().cp_attn_plan(None, 1, 2, 256, 64, 4, 0, C, 0.0) == -1
+    assert cp.lib().cp_attn_plan_destroy(None) == 0
+
+
+@pytest.mark.parametrize("S,N,layout,causal", [
+    (32768, 8, "zigzag", True), (32768, 8, "contiguous", True), (4096, 4, "zigzag", True),
+    (131072, 4, "zigzag", True), (131072, 4, "contiguous", True), (256, 4, "contiguous", False),
+    (800, 4, "contiguous", True), (384, 3, "zigzag", True), (1000, 5, "zigzag", True),
+])
+def test_plan_tile_counts_match_oracle(S, N, layout, causal):
+    B, H = 2, 3
+    plan = cp.Plan(B, H, S, 128, N, causal, layout)
+    per_rank, total = plan.tile_counts()
+    ref = Sch.tile_pair_counts(S, N, layout, causal) * B * H
+    assert per_rank == [int(x) for x in ref]
+    assert total == int(ref.sum())
+    plan.close()
+
+
+def test_plan_zigzag_balance_and_contiguous_imbalance():
+    w = WORKLOADS["zigzag_32k"]
+    z = cp.Plan(w.B, w.H, w.S, w.D, w.N, True, "zigzag").tile_counts()[0]
+    c = cp.Plan(w.B, w.H, w.S, w.D, w.N, True, "contiguous").tile_counts()[0]
+    assert len(set(z)) == 1 and z[0] == 4112 * w.H
+    assert abs(max(c) / (sum(c) / len(c)) - 1.8716) < 1e-4
+
+
+def test_workspace_and_map_sizes():
+    p = cp.Plan(2, 32, 16384, 128, 8, False, "ulysses")
+    assert p.workspace_bytes(False) == 4 * 2 * 16384 * 32 * 128 * 2
+    assert p.index_map_len() == 8 * 2 * 16384
+    assert p.tile_counts()[0] == [2 * 4 * 128 * 128] * 8
+    z = cp.Plan(1, 16, 4096, 128, 4, True, "zigzag")
+    assert z.workspace_bytes(False) == 0 and z.workspace_bytes(True) == 0
+    assert z.index_map_len() == 4096
+    assert z.num_items() == 4 * 16 * 4     # ranks x heads x query-tile pairs (T=1024)
