@@ -1,0 +1,359 @@
+"""Benchmark of context-parallel attention on B200: one JSON line on rank 0.
+
+A step is one pass of the hot path over one batch of the 32k zigzag workload
+(B=1, H=32, S=32768, D=128, 8 virtual ranks, causal), starting from Q/K/V in
+natural [B, S, H, D] layout resident in HBM:
+  1. layout map: Q, K, V natural -> zigzag rank-major (index-mapped copy kernel);
+  2. fused context-parallel attention (ring-order key walk, online-softmax
+     merge, causal tile skipping) writing O and lse;
+  3. layout map: O rank-major -> natural.
+``value`` counts the metric's FLOPs (4*B*H*S^2*D / 2 for causal) per step.
+The attention kernel alone is timed on its own stream for the roofline; the
+unfused path (per-step partials + merge kernel) is timed as a component.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+Under torchrun every rank runs its own replica of the workload (independent
+problems, no data-path collective: weak scaling) and rank 0 prints the line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "causal CP-attention fwd TFLOP/s and % of B200 BF16 dense peak, 1 GPU"
+WORKLOAD = "zigzag_32k"
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for ln in open(self.path):
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        mx = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [x for x in sm if x > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+                if any(r[3].replace(".", "").isdigit() for r in rows) else None}
+
+
+def oracle_sample_rate(w, max_rows: int, budget_s: float):
+    """Time the CPU oracle on sampled rows of the workload: (TFLOP/s, rows, seconds, cores)."""
+    import numpy as np
+    from oracle import attention as A
+    from workloads import make_qkv, sample_rows
+    q, k, v = make_qkv(w)
+    rows = sample_rows(w)
+    rng = np.random.default_rng(0)
+    rows = rows[rng.permutation(len(rows))[:max_rows]]
+    f = lambda t: t.float().numpy()
+    qn, kn, vn = f(q), f(k), f(v)
+    cores = len(os.sched_getaffinity(0))
+    done, flops, t0 = 0, 0.0, time.perf_counter()
+    chunk = 128
+    while done < len(rows) and time.perf_counter() - t0 < budget_s:
+        sel = rows[done:done + chunk]
+        A.attention_rows(qn, kn, vn, sel, causal=w.causal)
+        keys = (sel[:, 2] + 1) if w.causal else np.full(len(sel), w.S)
+        flops += float((4.0 * w.D * keys).sum())
+        done += len(sel)
+    dt = time.perf_counter() - t0
+    return flops / dt / 1e12, done, dt, cores
+
+
+def run_reference(args):
+    """The reference arm: the fp64 CPU oracle, as it stands, on bounded samples."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from workloads import WORKLOADS
+    w = WORKLOADS[WORKLOAD]
+    per_step = 12.0
+    rates, secs = [], []
+    for i in range(args.warmup + args.steps):
+        tf, rows, dt, cores = oracle_sample_rate(w, max_rows=4096, budget_s=per_step)
+        if i >= args.warmup:
+            rates.append(tf)
+            secs.append(dt)
+    value = statistics.median(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * statistics.median(secs),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "S": w.S, "D": w.D, "N": w.N,
+                                        "causal": w.causal, "layout": w.layout},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"up to 4096 seeded sampled query rows per step, {per_step:.0f} s budget; "
+                                   f"throughput counted as 4*D*(allowed keys) per row"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import context_long_sequence_cp_b200 as cp
+    from workloads import WORKLOADS, make_qkv
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = WORKLOADS[WORKLOAD]
+    B, H, S, D, N = w.B, w.H, w.S, w.D, w.N
+    plan = cp.Plan(B, H, S, D, N, w.causal, w.layout)
+    q_h, k_h, v_h = make_qkv(w)                       # natural, bf16, host
+    q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
+    qz, kz, vz, oz = (torch.empty_like(q).view(N, B, S // N, H, D) for _ in range(4))
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, S, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        cp.layout_permute(plan, q, 0, out=qz)
+        cp.layout_permute(plan, k, 0, out=kz)
+        cp.layout_permute(plan, v, 0, out=vz)
+        cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=lse)
+        cp.layout_permute(plan, oz, 1, out=o)
+
+    launches_per_step = 5
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x: float) -> float:
+        if ws == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    st = cp.check(plan)
+    if st != 0:
+        raise RuntimeError(f"warm-up failed: {cp.status_string(st)}")
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        barrier()
+    st = cp.check(plan)
+    if st != 0:
+        raise RuntimeError(f"timed run failed: {cp.status_string(st)}")
+    ms = max_over_ranks(ev0.elapsed_time(ev1)) / args.steps
+    value = ws * w.flops / (ms * 1e-3) / 1e12
+
+    # --- attention kernel alone (dominant kernel), CUDA events on its stream
+    att_ms = []
+    for _ in range(max(5, args.steps)):
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=lse)
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        att_ms.append(a0.elapsed_time(a1))
+    att = statistics.median(att_ms)
+    att_tflops = w.flops / (att * 1e-3) / 1e12
+
+    # --- permute kernel alone (HBM-bound): 2 bytes read + 2 written per element
+    perm_ms = []
+    for _ in range(5):
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        cp.layout_permute(plan, q, 0, out=qz)
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        perm_ms.append(a0.elapsed_time(a1))
+    perm = statistics.median(perm_ms)
+    perm_gbs = 2 * q.numel() * 2 / (perm * 1e-3) / 1e9
+
+    # --- unfused path: per-step partials + merge kernel
+    op = torch.empty(N, plan.rows, D, dtype=torch.float32, device=dev)
+    lp = torch.empty(N, plan.rows, dtype=torch.float32, device=dev)
+    om = torch.empty(plan.rows, D, dtype=torch.bfloat16, device=dev)
+    lm = torch.empty(plan.rows, dtype=torch.float32, device=dev)
+    cp.attn_fwd_partials(plan, qz, kz, vz, o_parts=op, lse_parts=lp)
+    cp.merge_partials(op, lp, o_out=om, lse_out=lm)
+    torch.cuda.synchronize(dev)
+    m0, m1, m2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    m0.record(stream)
+    cp.attn_fwd_partials(plan, qz, kz, vz, o_parts=op, lse_parts=lp)
+    m1.record(stream)
+    cp.merge_partials(op, lp, o_out=om, lse_out=lm)
+    m2.record(stream)
+    torch.cuda.synchronize(dev)
+    part_ms, merge_ms = m0.elapsed_time(m1), m1.elapsed_time(m2)
+    nonempty = int(torch.isfinite(lp).sum().item())
+    merge_bytes = nonempty * (4 * D + 4) + (N * plan.rows - nonempty) * 4 + plan.rows * (2 * D + 4)
+    merge_gbs = merge_bytes / (merge_ms * 1e-3) / 1e9
+    if cp.check(plan) != 0:
+        raise RuntimeError("component runs failed")
+
+    # --- end to end through the public API from pinned host buffers
+    q_p, k_p, v_p = (x.pin_memory() for x in (q_h, k_h, v_h))
+    o_p = torch.empty_like(q_h).pin_memory()
+    lse_p = torch.empty(B, H, S, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        q.copy_(q_p, non_blocking=True)
+        k.copy_(k_p, non_blocking=True)
+        v.copy_(v_p, non_blocking=True)
+        step()
+        o_p.copy_(o, non_blocking=True)
+        lse_p.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(3, min(args.steps, 10))
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e_ms = max_over_ranks(e0.elapsed_time(e1)) / e_steps
+    e2e_value = ws * w.flops / (e_ms * 1e-3) / 1e12
+    h2d = 3 * q.numel() * 2
+    d2h = o.numel() * 2 + lse.numel() * 4
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "attn_fwd_zigzag_32k_traffic.json")
+    if os.path.exists(prof):
+        with open(prof) as f:
+            traffic = json.load(f).get("dram_bytes_per_launch")
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "H": H, "S": S, "D": D, "N": N, "causal": w.causal,
+                   "layout": w.layout, "flops_per_step": w.flops,
+                   "l2": "inputs larger than L2 (3 x 256 MiB of Q/K/V read per step)",
+                   "step": "permute Q,K,V natural->zigzag; fused CP attention; permute O back"},
+        "roofline": {"kernel": "attn_fwd_kernel<128,false>", "bound": "tensor", "achieved": att_tflops,
+                     "peak": peak, "unit": "TFLOP/s", "frac": att_tflops / peak, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
+                     "frac_of_nominal_2250": att_tflops / NOMINAL_BF16_TFLOPS, "ms": att},
+        "components": {
+            "attention_ms": att, "attention_tflops": att_tflops,
+            "permute_ms": perm, "permute_gbs": perm_gbs, "permute_frac_hbm": perm_gbs / float(peaks["hbm_gbs"]),
+            "partials_ms": part_ms, "merge_ms": merge_ms, "merge_gbs": merge_gbs,
+            "merge_frac_hbm": merge_gbs / float(peaks["hbm_gbs"]),
+            "unfused_tflops": w.flops / ((part_ms + merge_ms) * 1e-3) / 1e12,
+        },
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        tf, rows, dt, cores = oracle_sample_rate(w, max_rows=4096, budget_s=15.0)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                "sample": f"{rows} seeded sampled query rows of {WORKLOAD} in {dt:.1f} s "
+                                          f"(fp64 NumPy); FLOPs counted as 4*D*(allowed keys) per row"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    plan.close()
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

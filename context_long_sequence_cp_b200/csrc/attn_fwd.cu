@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_drain(smem_addr(&sm.drain), 0, p.wait_limit_ns);
       }
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax warpgroups
     const int wg = warp >> 2;
     const int quad = warp & 3;
