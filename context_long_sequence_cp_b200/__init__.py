@@ -40,7 +40,12 @@ SIGNATURES = {
     "cp_attn_check": (_I, [_P, _P]),
     "cp_status_string": (ctypes.c_char_p, [_I]),
     "cp_debug_wait_timeout_probe": (_I, [_P, _I, _P]),
+    "cp_attn_fwd_ulysses_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P]),
 }
+
+# Size of the library's fixed device scratch used by the no-alloc Ulysses
+# forward (CP_NOALLOC_SCRATCH_BYTES in include/cp_attn.h).
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class CpAttnError(RuntimeError):
@@ -194,6 +199,20 @@ def check(plan: Plan, stream=None) -> int:
 def debug_wait_timeout_probe(plan: Plan, timeout_us: int, stream=None):
     _check("cp_debug_wait_timeout_probe",
            lib().cp_debug_wait_timeout_probe(plan.handle, int(timeout_us), _stream(stream)))
+
+
+def attn_fwd_ulysses_noalloc(plan: Plan, q, k, v, o, lse=None, stream=None):
+    """Ulysses forward that allocates nothing (``cp_attn_fwd_ulysses_noalloc``).
+
+    For callers that cannot allocate device memory at call time: the head-group
+    copies live in the library's fixed 32 MiB device scratch instead of a
+    workspace, so ``o`` (and ``lse`` if wanted) must be passed in. Calls that
+    may overlap on the GPU share that scratch and must be serialised.
+    """
+    _check("cp_attn_fwd_ulysses_noalloc",
+           lib().cp_attn_fwd_ulysses_noalloc(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                            _stream(stream)))
+    return o, lse
 
 
 def status_string(status: int) -> str:

@@ -377,3 +377,29 @@ int cp_debug_wait_timeout_probe(cp_attn_plan_t plan, int timeout_us, cp_stream_t
 }
 
 }  // extern "C"
+
+// Ulysses forward on a caller-chosen scratch buffer: the same launches as the
+// Ulysses branch of cp_attn_fwd, with the head-group copies placed in `scratch`.
+int cp_internal_ulysses_fwd_scratch(cp_attn_plan_s* plan, const void* q, const void* k, const void* v, void* o,
+                                    float* lse, void* scratch, size_t scratch_bytes, cudaStream_t st) {
+  if (plan == nullptr || q == nullptr || k == nullptr || v == nullptr || o == nullptr) return CP_ERR_INVALID_ARG;
+  if (plan->layout != CP_LAYOUT_ULYSSES) return CP_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(scratch))
+    return CP_ERR_ALIGNMENT;
+  const size_t tensor = static_cast<size_t>(plan->B) * plan->S * plan->H * plan->D * 2;
+  if (scratch == nullptr || scratch_bytes < 4 * tensor) return CP_ERR_WORKSPACE;
+  int rc = ensure_device(plan);
+  if (rc != CP_OK) return rc;
+  char* ws = static_cast<char*>(scratch);
+  void* gq = ws;
+  void* gk = ws + tensor;
+  void* gv = ws + 2 * tensor;
+  void* go = ws + 3 * tensor;
+  const PermuteArgs fwd = permute_args(plan, 0, 2);
+  if (launch_permute(fwd, q, gq, st) != cudaSuccess || launch_permute(fwd, k, gk, st) != cudaSuccess ||
+      launch_permute(fwd, v, gv, st) != cudaSuccess)
+    return CP_ERR_CUDA;
+  rc = launch_view(plan, plan->g, gq, gk, gv, go, lse, nullptr, nullptr, 0, 1, false, st);
+  if (rc != CP_OK) return rc;
+  return launch_permute(permute_args(plan, 1, 2), go, o, st) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}

@@ -55,3 +55,14 @@ cudaError_t launch_index_map(const PermuteArgs& a, int64_t* map_out, cudaStream_
 cudaError_t launch_wait_probe(int* status, uint64_t limit_ns, cudaStream_t stream);
 
 }  // namespace cpattn
+
+// api.cu: the Ulysses forward with a caller-chosen scratch buffer of at least
+// cp_attn_workspace_bytes(plan, 0) bytes (used by the no-alloc entry point).
+struct cp_attn_plan_s;
+int cp_internal_ulysses_fwd_scratch(cp_attn_plan_s* plan, const void* q, const void* k, const void* v,
+                                    void* o, float* lse, void* scratch, size_t scratch_bytes,
+                                    cudaStream_t stream);
+
+namespace cpattn {
+
+}  // namespace cpattn

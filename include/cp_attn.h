@@ -217,6 +217,45 @@ CP_API const char* cp_status_string(int status);
  */
 CP_API int cp_debug_wait_timeout_probe(cp_attn_plan_t plan, int timeout_us, cp_stream_t stream);
 
+/*
+ * Ulysses forward that allocates nothing (no counterpart on the pages: this is
+ * an interface convenience of this library, not part of the method).
+ *
+ * Who needs it: callers that must not call cudaMalloc at the point of the
+ * call -- code whose device memory is owned by another allocator (a framework
+ * caching allocator that would otherwise have to hand out a multi-megabyte
+ * workspace), code that runs where allocation is forbidden or would
+ * synchronise the device (a latency-critical loop), or code that simply has
+ * no way to obtain a workspace buffer. cp_attn_fwd's Ulysses path needs
+ * 4*B*S*H*D*2 bytes of workspace for the head-group copies of Q, K, V and O;
+ * this variant takes them from a fixed scratch array that the library holds
+ * in device memory instead.
+ *
+ * Same arguments and results as cp_attn_fwd for a CP_LAYOUT_ULYSSES plan,
+ * minus the workspace: q, k, v, o are sequence shards [N][B][S/N][H][D] bf16,
+ * lse is float32 [B][H][S] (may be NULL); the plan itself must have been
+ * created beforehand (cp_attn_plan allocates its small work-list table once).
+ *
+ * Limits and behaviour:
+ *   - The scratch is a static device array of CP_NOALLOC_SCRATCH_BYTES
+ *     (32 MiB). Every GPU on which the library's kernels are loaded holds it
+ *     until the process exits. Plans needing more (4*B*S*H*D*2 bytes) are
+ *     rejected with CP_ERR_WORKSPACE before anything is launched; plans of
+ *     another layout with CP_ERR_UNSUPPORTED.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture on that device.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents. Nothing in it has to start at zero: each call writes every
+ *     byte it reads. Two calls whose work can overlap on the GPU (different
+ *     streams without ordering, or different host threads) race on it:
+ *     serialise them.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define CP_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+CP_API int cp_attn_fwd_ulysses_noalloc(cp_attn_plan_t plan, const void* q, const void* k, const void* v,
+                                       void* o, float* lse, cp_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
