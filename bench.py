@@ -165,6 +165,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="only launch the fused attention kernel warmup+steps times (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -214,6 +216,15 @@ def main():
         t = torch.tensor([x], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
+
+    if args.profile:
+        for x, y in ((q, qz), (k, kz), (v, vz)):
+            cp.layout_permute(plan, x, 0, out=y)
+        for _ in range(args.warmup + args.steps):
+            cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=lse)
+        st = cp.check(plan)
+        print(json.dumps({"profile": "attn_fwd", "launches": args.warmup + args.steps, "status": st}))
+        return 0 if st == 0 else 1
 
     for _ in range(args.warmup):
         step()
@@ -314,8 +325,18 @@ def main():
     traffic = None
     prof = os.path.join(ROOT, "profiles", "attn_fwd_zigzag_32k_traffic.json")
     if os.path.exists(prof):
+        # DRAM bytes of one launch from an ncu capture, valid only for the kernel
+        # source it was taken on (null once the kernel changed).
+        import hashlib
+        csrc = os.path.join(ROOT, "context_long_sequence_cp_b200", "csrc")
+        h = hashlib.sha256()
+        for name in ("attn_fwd.cu", "sm100.cuh", "geometry.h"):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
         with open(prof) as f:
-            traffic = json.load(f).get("dram_bytes_per_launch")
+            rec = json.load(f)
+        if rec.get("source_sha256_16") == h.hexdigest()[:16]:
+            traffic = rec.get("dram_bytes_per_launch")
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
