@@ -28,6 +28,13 @@ struct cp_attn_plan_s {
   WorkItem* d_items = nullptr;      // device copy of the work list
   int* d_status = nullptr;          // device status word
   int device = -1;
+  // Precomputed key walks per query-tile pair (rank, qp): entries in ring order
+  // and the offset of every ring step (NR + 1 offsets per pair).
+  int npairs = 0;
+  std::vector<int> step_off;
+  std::vector<uint32_t> entries;
+  int* d_step_off = nullptr;
+  uint32_t* d_entries = nullptr;
 };
 
 namespace {
@@ -102,6 +109,9 @@ int launch_view(cp_attn_plan_s* p, const Geometry& g, const void* q, const void*
   P.scale_log2 = p->scale * 1.4426950408889634f;
   P.items = p->d_items;
   P.n_items = static_cast<int>(p->items.size());
+  P.step_off = p->d_step_off;
+  P.entries = p->d_entries;
+  P.npairs = p->npairs;
   P.o = static_cast<__nv_bfloat16*>(o);
   P.lse = lse;
   P.lse_B = p->lse_B;
@@ -147,6 +157,9 @@ int cp_attn_plan(cp_attn_plan_t* out, int B, int H, int S, int D, int N, int cau
   // int32 indexing limits of the kernels: tokens per view, view row blocks, TMA dims.
   if (static_cast<int64_t>(B) * N > (1 << 20) || static_cast<int64_t>(B) * S * H * D > (int64_t(1) << 40))
     return CP_ERR_UNSUPPORTED;
+  // Packed walk entries: key rank < 2^12, key tile index < 2^13.
+  if (N >= (1 << kEntryRankBits) || (static_cast<int64_t>(S) + kTile - 1) / kTile >= (1 << kEntryTileBits))
+    return CP_ERR_UNSUPPORTED;
 
   cp_attn_plan_s* p = new (std::nothrow) cp_attn_plan_s();
   if (p == nullptr) return CP_ERR_INVALID_ARG;
@@ -169,8 +182,29 @@ int cp_attn_plan(cp_attn_plan_t* out, int B, int H, int S, int D, int N, int cau
                  causal};
   }
 
-  // Work list: every (rank, batch, head, query-tile pair) with its executed key tiles.
+  // Key walks: for every (rank, query-tile pair), the executed key tiles in ring
+  // order with both query tiles' classes, and where each ring step starts.
   const int npairs = (g.T + kPair - 1) / kPair;
+  p->npairs = npairs;
+  p->step_off.reserve(static_cast<size_t>(g.NR) * npairs * (g.NR + 1));
+  for (int r = 0; r < g.NR; ++r) {
+    for (int qp = 0; qp < npairs; ++qp) {
+      for (int t = 0; t < g.NR; ++t) {
+        p->step_off.push_back(static_cast<int>(p->entries.size()));
+        KeyTileWalk w;
+        w.init(g, r, qp * kPair, t, t + 1);
+        int rk, kt, c0, c1;
+        while (w.next(rk, kt, c0, c1)) p->entries.push_back(pack_entry(rk, kt, c0, c1));
+      }
+      p->step_off.push_back(static_cast<int>(p->entries.size()));
+    }
+  }
+  if (p->entries.size() >= (size_t(1) << 31)) {
+    delete p;
+    return CP_ERR_UNSUPPORTED;
+  }
+
+  // Work list: every (rank, batch, head, query-tile pair) with its executed key tiles.
   p->tile_counts.assign(N, 0);
   p->items.reserve(static_cast<size_t>(g.NR) * g.B * g.Hh * npairs);
   for (int r = 0; r < g.NR; ++r) {
@@ -200,15 +234,26 @@ int cp_attn_plan(cp_attn_plan_t* out, int B, int H, int S, int D, int N, int cau
   if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0) {
     cudaGetDevice(&p->device);
     const size_t bytes = p->items.size() * sizeof(WorkItem);
+    const size_t off_bytes = p->step_off.size() * sizeof(int);
+    const size_t ent_bytes = p->entries.size() * sizeof(uint32_t);
     bool ok = cudaMalloc(&p->d_items, bytes > 0 ? bytes : sizeof(WorkItem)) == cudaSuccess &&
               cudaMalloc(&p->d_status, sizeof(int)) == cudaSuccess &&
+              cudaMalloc(&p->d_step_off, off_bytes) == cudaSuccess &&
+              cudaMalloc(&p->d_entries, ent_bytes > 0 ? ent_bytes : sizeof(uint32_t)) == cudaSuccess &&
               cudaMemcpy(p->d_items, p->items.data(), bytes, cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMemcpy(p->d_step_off, p->step_off.data(), off_bytes, cudaMemcpyHostToDevice) == cudaSuccess &&
+              (ent_bytes == 0 ||
+               cudaMemcpy(p->d_entries, p->entries.data(), ent_bytes, cudaMemcpyHostToDevice) == cudaSuccess) &&
               cudaMemset(p->d_status, 0, sizeof(int)) == cudaSuccess;
     if (!ok) {
       cudaFree(p->d_items);
       cudaFree(p->d_status);
+      cudaFree(p->d_step_off);
+      cudaFree(p->d_entries);
       p->d_items = nullptr;
       p->d_status = nullptr;
+      p->d_step_off = nullptr;
+      p->d_entries = nullptr;
     }
   } else {
     cudaGetLastError();   // clear the "no device" error
@@ -221,6 +266,8 @@ int cp_attn_plan_destroy(cp_attn_plan_t plan) {
   if (plan == nullptr) return CP_OK;
   if (plan->d_items != nullptr) cudaFree(plan->d_items);
   if (plan->d_status != nullptr) cudaFree(plan->d_status);
+  if (plan->d_step_off != nullptr) cudaFree(plan->d_step_off);
+  if (plan->d_entries != nullptr) cudaFree(plan->d_entries);
   delete plan;
   return CP_OK;
 }

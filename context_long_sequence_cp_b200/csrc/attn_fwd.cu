@@ -48,13 +48,20 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows by > 256x
+// In full tiles, one column pair in kPolyEvery takes its exponentials on the FMA
+// pipe (ex2_poly) instead of the MUFU unit; 0 keeps every exponential on MUFU.
+#ifndef CP_POLY_EVERY
+#define CP_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = CP_POLY_EVERY;
+
 
 template <int D>
 struct Cfg {
   static constexpr int kTileBytes = kTile * D * 2;               // one 128 x D bf16 tile
   static constexpr int kBlocks = D / 64;                         // 128-byte column blocks
   static constexpr int kBlockBytes = kTile * 128;                // 16 KB
-  static constexpr int kStages = D == 128 ? 4 : 6;
+  static constexpr int kStages = D == 128 ? 5 : 8;
   static constexpr int kTmemCols = 512;
   static constexpr int kOCol = 256;
   static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);   // Q K^T, both K-major
@@ -148,6 +155,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = sm.tmem_base;
   WaitCtl ctl{&sm.abort, p.status, p.wait_limit_ns};
 
+  // Every role walks the same precomputed key list of each work item.
+  const int nstep_off = g.NR + 1;
+
   if (warp == 9) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -161,6 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rq = w.rb / g.B;
         const int bv = w.rb - rq * g.B;
         const int q0 = w.qp * kPair;
+        const int* off = p.step_off + (rq * p.npairs + w.qp) * nstep_off;
+        const int e_begin = __ldg(off + p.t_begin), e_end = __ldg(off + p.t_end);
         if (q_iter > 0) ok = mbar_wait(smem_addr(&sm.q_empty), (q_iter - 1) & 1, ctl);
         if (!ok) break;
         const uint32_t qbar = smem_addr(&sm.q_full);
@@ -170,11 +182,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(smem_addr(&sm.q[i][0]) + blk * C::kBlockBytes, &tm_q, qbar, blk * 64, w.h,
                         q0 + i * kTile, w.rb, pol_q);
         ++q_iter;
-        KeyTileWalk walk;
-        walk.init(g, rq, q0, p.t_begin, p.t_end);
-        int rk, kt, c0, c1;
-        while (ok && walk.next(rk, kt, c0, c1)) {
-          const int rbk = rk * g.B + bv;
+        for (int e = e_begin; e < e_end && ok; ++e) {
+          const uint32_t ent = __ldg(p.entries + e);
+          const int rbk = entry_rank(ent) * g.B + bv;
+          const int k0 = entry_tile(ent) * kTile;
           for (int which = 0; which < 2; ++which) {
             const int stage = kv_idx % C::kStages;
             const int round = kv_idx / C::kStages;
@@ -184,8 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(bar, C::kTileBytes);
             const CUtensorMap* map = which == 0 ? &tm_k : &tm_v;
             for (int blk = 0; blk < C::kBlocks; ++blk)
-              tma_load_4d(smem_addr(&sm.kv[stage][0]) + blk * C::kBlockBytes, map, bar, blk * 64,
-                          w.h, kt * kTile, rbk, pol_kv);
+              tma_load_4d(smem_addr(&sm.kv[stage][0]) + blk * C::kBlockBytes, map, bar, blk * 64, w.h, k0,
+                          rbk, pol_kv);
             ++kv_idx;
           }
         }
@@ -211,98 +222,94 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
         const WorkItem w = p.items[it];
         const int rq = w.rb / g.B;
-        const int q0 = w.qp * kPair;
-        // Count the PV products of each query tile so the last one can signal o_done.
-        int n_pv0 = 0, n_pv1 = 0;
-        {
-          KeyTileWalk cnt;
-          cnt.init(g, rq, q0, p.t_begin, p.t_end);
-          int rk, kt, c0, c1;
-          while (cnt.next(rk, kt, c0, c1)) {
-            n_pv0 += c0 != kSkip;
-            n_pv1 += c1 != kSkip;
-          }
+        const int* off = p.step_off + (rq * p.npairs + w.qp) * nstep_off;
+        const int e_begin = __ldg(off + p.t_begin), e_end = __ldg(off + p.t_end);
+        // The last PV of each query tile signals o_done: find where they are.
+        int last0 = -1, last1 = -1;
+        for (int e = e_begin; e < e_end; ++e) {
+          const uint32_t ent = __ldg(p.entries + e);
+          if (entry_c0(ent) != kSkip) last0 = e;
+          if (entry_c1(ent) != kSkip) last1 = e;
         }
         ok = mbar_wait(smem_addr(&sm.q_full), q_iter & 1, ctl);
         if (!ok) break;
         ++q_iter;
         tc_fence_after();
-        KeyTileWalk walk;
-        walk.init(g, rq, q0, p.t_begin, p.t_end);
-        int rk, kt, cur0, cur1;
-        if (!walk.next(rk, kt, cur0, cur1)) {
+        if (e_begin == e_end) {
           umma_commit(smem_addr(&sm.q_empty));
           continue;
         }
-        // First key tile: both S products.
+        // First key tile: its S products.
+        uint32_t cur = __ldg(p.entries + e_begin);
         int kst = kv_idx % C::kStages;
         ok = mbar_wait(smem_addr(&sm.kv_full[kst]), (kv_idx / C::kStages) & 1, ctl);
         if (!ok) break;
         ++kv_idx;
         tc_fence_after();
-        const uint32_t k_addr0 = smem_addr(&sm.kv[kst][0]);
-        if (cur0 != kSkip) {
-          issue_s<D>(tS0, q_addr0, k_addr0);
-          umma_commit(smem_addr(&sm.s_full[0]));
-        }
-        if (cur1 != kSkip) {
-          issue_s<D>(tS1, q_addr1, k_addr0);
-          umma_commit(smem_addr(&sm.s_full[1]));
+        {
+          const uint32_t k_addr = smem_addr(&sm.kv[kst][0]);
+          if (entry_c0(cur) != kSkip) {
+            issue_s<D>(tS0, q_addr0, k_addr);
+            umma_commit(smem_addr(&sm.s_full[0]));
+          }
+          if (entry_c1(cur) != kSkip) {
+            issue_s<D>(tS1, q_addr1, k_addr);
+            umma_commit(smem_addr(&sm.s_full[1]));
+          }
         }
         issued = true;
         umma_commit(smem_addr(&sm.kv_empty[kst]));
-        int seen0 = 0, seen1 = 0;
-        for (;;) {
-          int nrk, nkt, nxt0, nxt1;
-          const bool has_next = walk.next(nrk, nkt, nxt0, nxt1);
+        bool acc0 = false, acc1 = false;
+        for (int e = e_begin; e < e_end; ++e) {
+          const bool has_next = e + 1 < e_end;
+          const uint32_t nxt = has_next ? __ldg(p.entries + e + 1) : 0u;
+          // Both operand tiles of this step first (V of this tile, K of the next),
+          // so that once P is ready the PV and the next S issue back to back.
           const int vst = kv_idx % C::kStages;
           ok = mbar_wait(smem_addr(&sm.kv_full[vst]), (kv_idx / C::kStages) & 1, ctl);
           if (!ok) break;
           ++kv_idx;
-          tc_fence_after();
-          const uint32_t v_addr = smem_addr(&sm.kv[vst][0]);
           int nst = 0;
-          uint32_t nk_addr = 0;
-          // Query tile 0: PV0(cur), then S0(next).
-          if (cur0 != kSkip) {
-            ok = mbar_wait(smem_addr(&sm.p_full[0]), p_cnt0 & 1, ctl);
-            if (!ok) break;
-            ++p_cnt0;
-            tc_fence_after();
-            issue_pv<D>(tO0, tS0, v_addr, seen0 > 0);
-            if (++seen0 == n_pv0) umma_commit(smem_addr(&sm.o_done[0]));
-          }
           if (has_next) {
             nst = kv_idx % C::kStages;
             ok = mbar_wait(smem_addr(&sm.kv_full[nst]), (kv_idx / C::kStages) & 1, ctl);
             if (!ok) break;
             ++kv_idx;
+          }
+          tc_fence_after();
+          const uint32_t v_addr = smem_addr(&sm.kv[vst][0]);
+          const uint32_t nk_addr = smem_addr(&sm.kv[nst][0]);
+          // Query tile 0: PV0(cur), then S0(next).
+          if (entry_c0(cur) != kSkip) {
+            ok = mbar_wait(smem_addr(&sm.p_full[0]), p_cnt0 & 1, ctl);
+            if (!ok) break;
+            ++p_cnt0;
             tc_fence_after();
-            nk_addr = smem_addr(&sm.kv[nst][0]);
-            if (nxt0 != kSkip) {
-              issue_s<D>(tS0, q_addr0, nk_addr);
-              umma_commit(smem_addr(&sm.s_full[0]));
-            }
+            issue_pv<D>(tO0, tS0, v_addr, acc0);
+            acc0 = true;
+            if (e == last0) umma_commit(smem_addr(&sm.o_done[0]));
+          }
+          if (has_next && entry_c0(nxt) != kSkip) {
+            issue_s<D>(tS0, q_addr0, nk_addr);
+            umma_commit(smem_addr(&sm.s_full[0]));
           }
           // Query tile 1: PV1(cur), then S1(next).
-          if (cur1 != kSkip) {
+          if (entry_c1(cur) != kSkip) {
             ok = mbar_wait(smem_addr(&sm.p_full[1]), p_cnt1 & 1, ctl);
             if (!ok) break;
             ++p_cnt1;
             tc_fence_after();
-            issue_pv<D>(tO1, tS1, v_addr, seen1 > 0);
-            if (++seen1 == n_pv1) umma_commit(smem_addr(&sm.o_done[1]));
+            issue_pv<D>(tO1, tS1, v_addr, acc1);
+            acc1 = true;
+            if (e == last1) umma_commit(smem_addr(&sm.o_done[1]));
           }
-          if (has_next && nxt1 != kSkip) {
+          if (has_next && entry_c1(nxt) != kSkip) {
             issue_s<D>(tS1, q_addr1, nk_addr);
             umma_commit(smem_addr(&sm.s_full[1]));
           }
-          if (!ok) break;
           if (has_next) umma_commit(smem_addr(&sm.kv_empty[nst]));
           umma_commit(smem_addr(&sm.kv_empty[vst]));
-          if (!has_next) break;
-          cur0 = nxt0;
-          cur1 = nxt1;
+          cur = nxt;
         }
         if (!ok) break;
         umma_commit(smem_addr(&sm.q_empty));
@@ -323,6 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tbase + lane_off + wg * 128;
     const uint32_t tO = tbase + lane_off + C::kOCol + wg * D;
     const float sl2 = p.scale_log2;
+    const int cls_shift = wg == 0 ? 25 : 27;
     int s_cnt = 0, od_cnt = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
@@ -333,19 +341,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tl = q_first + wg * kTile + row;
       const bool valid = tl < g.T;
       const int64_t gq = global_pos(g, rq, valid ? tl : g.T - 1);
+      const int* off = p.step_off + (rq * p.npairs + w.qp) * nstep_off;
+      const int e_begin = __ldg(off + p.t_begin), e_end = __ldg(off + p.t_end);
       float m_run = -INFINITY, l_run = 0.f;
       int ntile = 0;
-      KeyTileWalk walk;
-      walk.init(g, rq, q_first, p.t_begin, p.t_end);
-      int rk, kt, c0, c1;
-      while (walk.next(rk, kt, c0, c1)) {
-        const int cls = wg == 0 ? c0 : c1;
+      uint32_t ent = e_begin < e_end ? __ldg(p.entries + e_begin) : 0u;
+      for (int e = e_begin; e < e_end; ++e) {
+        const uint32_t cur = ent;
+        if (e + 1 < e_end) ent = __ldg(p.entries + e + 1);   // prefetch the next entry
+        const int cls = static_cast<int>((cur >> cls_shift) & 3u);
         if (cls == kSkip) continue;
         ok = mbar_wait(smem_addr(&sm.s_full[wg]), s_cnt & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
+        const int rk = entry_rank(cur);
+        const int kt = entry_tile(cur);
         float s[kTile];
         tmem_ld128(tS, reinterpret_cast<uint32_t*>(s));
         if (cls == kMasked) {
@@ -353,9 +365,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < kTile; ++j) s[j] = j < lim ? s[j] : -INFINITY;
         }
-        float mx = s[0];
+        // Row max: four independent chains of 3-input maxima (short dependency chains).
+        float mx;
+        {
+          float mc[4];
 #pragma unroll
-        for (int j = 1; j < kTile; ++j) mx = fmaxf(mx, s[j]);
+          for (int c = 0; c < 4; ++c) {
+            float m = s[32 * c];
+#pragma unroll
+            for (int j = 1; j + 1 < 32; j += 2) m = max3(m, s[32 * c + j], s[32 * c + j + 1]);
+            mc[c] = fmaxf(m, s[32 * c + 31]);
+          }
+          mx = fmaxf(max3(mc[0], mc[1], mc[2]), mc[3]);
+        }
         const float m_tile = mx * sl2;
         const float m_new = fmaxf(m_run, m_tile);
         const bool resc = m_new - m_run > kRescaleThreshold;   // false while both are -inf
@@ -366,19 +388,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_run *= alpha;
         }
         const float m_use = m_run == -INFINITY ? 0.f : m_run;
-        float lsum = 0.f;
+        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (cls == kMasked) {
+          // Masked tiles: every exponential on the MUFU unit, so -inf gives exactly 0.
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float e0 = ex2_approx(fmaf(s[c * 32 + 2 * j], sl2, -m_use));
-            const float e1 = ex2_approx(fmaf(s[c * 32 + 2 * j + 1], sl2, -m_use));
-            lsum += e0 + e1;
-            pk[j] = pack_bf16x2(e0, e1);
+            for (int j = 0; j < 16; ++j) {
+              const float e0 = ex2_approx(fmaf(s[c * 32 + 2 * j], sl2, -m_use));
+              const float e1 = ex2_approx(fmaf(s[c * 32 + 2 * j + 1], sl2, -m_use));
+              ls[j & 7] += e0 + e1;
+              pk[j] = pack_bf16x2(e0, e1);
+            }
+            tmem_st16(tS + c * 16, pk);
           }
-          tmem_st16(tS + c * 16, pk);
+        } else {
+          // Full tiles: one column pair in kPolyEvery takes its exponentials on the FMA pipe.
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float x0 = fmaf(s[c * 32 + 2 * j], sl2, -m_use);
+              const float x1 = fmaf(s[c * 32 + 2 * j + 1], sl2, -m_use);
+              const bool poly = kPolyEvery > 0 && (j % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+              const float e0 = poly ? ex2_poly(x0) : ex2_approx(x0);
+              const float e1 = poly ? ex2_poly(x1) : ex2_approx(x1);
+              ls[j & 7] += e0 + e1;
+              pk[j] = pack_bf16x2(e0, e1);
+            }
+            tmem_st16(tS + c * 16, pk);
+          }
         }
+        const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         if (ntile > 0 && __any_sync(0xffffffffu, resc)) {
           // O holds the previous PV products (complete: this tile's s_full was
           // committed after them) and the next PV waits for p_full: rescale in place.

@@ -17,6 +17,11 @@ struct FwdParams {
   float scale_log2;            // softmax scale * log2(e)
   const WorkItem* items;       // device work list
   int n_items;
+  // Precomputed key walks: the walk of query-tile pair (rq, qp) over ring step t
+  // is entries[step_off[(rq*npairs + qp)*(NR+1) + t] .. step_off[... + t + 1]).
+  const int* step_off;
+  const uint32_t* entries;
+  int npairs;
   __nv_bfloat16* o;            // fused output, view layout [NR*B][T][Hh][D]
   float* lse;                  // natural [lse_B][lse_H][lse_S]; may be null
   int lse_B, lse_H;

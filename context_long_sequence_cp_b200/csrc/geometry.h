@@ -91,6 +91,20 @@ struct WorkItem {
   int cost;  // executed key tiles (both query tiles), used for ordering
 };
 
+// A precomputed key-tile entry of a work item's walk, packed in 32 bits:
+// bits [0,13) key tile index, [13,25) key rank, [25,27) class of query tile 0,
+// [27,29) class of query tile 1.
+constexpr int kEntryTileBits = 13;
+constexpr int kEntryRankBits = 12;
+CP_HD uint32_t pack_entry(int rk, int kt, int c0, int c1) {
+  return static_cast<uint32_t>(kt) | (static_cast<uint32_t>(rk) << kEntryTileBits) |
+         (static_cast<uint32_t>(c0) << 25) | (static_cast<uint32_t>(c1) << 27);
+}
+CP_HD int entry_tile(uint32_t e) { return static_cast<int>(e & ((1u << kEntryTileBits) - 1)); }
+CP_HD int entry_rank(uint32_t e) { return static_cast<int>((e >> kEntryTileBits) & ((1u << kEntryRankBits) - 1)); }
+CP_HD int entry_c0(uint32_t e) { return static_cast<int>((e >> 25) & 3u); }
+CP_HD int entry_c1(uint32_t e) { return static_cast<int>((e >> 27) & 3u); }
+
 // Walks the key tiles one work item visits, in ring order (t = t_begin..t_end-1,
 // key tiles ascending within each step), yielding the classes for both query
 // tiles and skipping pairs where both are kSkip. Causal masks make skips

@@ -297,6 +297,31 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 3-input maximum (sm_100 max.f32 with three sources).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x on the FMA/ALU pipes instead of the MUFU unit, for x <= 8.
+// Method: Cody-Waite style range reduction x = n + f, n = round(x) obtained by
+// adding 1.5 * 2^23 (the integer lands in the low mantissa bits, f in
+// [-1/2, 1/2]); 2^f by a degree-3 polynomial whose coefficients minimise the
+// maximum relative error on [-1/2, 1/2] (Remez exchange, fitted by
+// csrc/gen_exp2_poly.py: max relative error 7.5e-5); 2^n applied by adding n to
+// the exponent field. Inputs below -125 are clamped to -125 (result ~2^-125, not
+// 0): callers use it only where no -inf occurs.
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(5.517166853e-02f, f, 2.426111251e-01f), f, 6.932609677e-01f), f,
+                       9.999280572e-01f);
+  // (bits(t) << 23) == n << 23: the rounding constant's low 9 bits are zero.
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
