@@ -48,12 +48,8 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows by > 256x
-// In full tiles, one column pair in kPolyEvery takes its exponentials on the FMA
-// pipe (ex2_poly) instead of the MUFU unit; 0 keeps every exponential on MUFU.
-#ifndef CP_POLY_EVERY
-#define CP_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = CP_POLY_EVERY;
+// P is handed to the MMA warp in two halves (keys 0-63, 64-127), so the first
+// half of PV starts while the exponentials of the second half are computed.
 
 
 template <int D>
@@ -76,7 +72,7 @@ struct alignas(1024) Smem {
   uint64_t kv_full[Cfg<D>::kStages];
   uint64_t kv_empty[Cfg<D>::kStages];
   uint64_t s_full[2];
-  uint64_t p_full[2];
+  uint64_t p_full[2][2];   // [query tile][P half]
   uint64_t o_done[2];
   uint64_t drain;
   uint32_t tmem_base;
@@ -97,16 +93,37 @@ __device__ __forceinline__ void issue_s(uint32_t tS, uint32_t q_addr, uint32_t k
   }
 }
 
-template <int D>
+template <int D, int KK_BEGIN, int KK_END>
 __device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint32_t v_addr, bool accumulate) {
-  // O (+)= P V over K = 128 keys in steps of 16: P from TMEM (8 packed columns per
-  // step), V from shared memory as an MN-major operand (8-key groups 1024 B apart,
-  // 64-column blocks kBlockBytes apart).
+  // O (+)= P V over keys [16*KK_BEGIN, 16*KK_END) in steps of 16: P from TMEM (8
+  // packed columns per step), V from shared memory as an MN-major operand (8-key
+  // groups 1024 B apart, 64-column blocks kBlockBytes apart).
 #pragma unroll
-  for (int kk = 0; kk < kTile / 16; ++kk) {
+  for (int kk = KK_BEGIN; kk < KK_END; ++kk) {
     const uint64_t b = smem_desc_sw128(v_addr + kk * 2048, Cfg<D>::kBlockBytes, 1024);
     umma_ts(tO, tP + kk * 8, b, Cfg<D>::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
   }
+}
+
+// Exponentials of one 32-column chunk c of a score row, packed to bf16 pairs and
+// stored as 16 TMEM columns of P at tS + 16c; row-sum partials accumulate in ls.
+// The scaling x = s * scale - m runs two columns per instruction (f32x2).
+__device__ __forceinline__ void softmax_chunk(const float (&s)[kTile], int c, float sl2, float m_use,
+                                              uint32_t tS, float (&ls)[8]) {
+  uint32_t pk[16];
+  const uint64_t sl2_2 = f2_pack(sl2, sl2);
+  const uint64_t nm_2 = f2_pack(-m_use, -m_use);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int col = c * 32 + 2 * j;
+    float x0, x1;
+    f2_unpack(f2_fma(f2_pack(s[col], s[col + 1]), sl2_2, nm_2), x0, x1);
+    const float e0 = ex2_approx(x0);
+    const float e1 = ex2_approx(x1);
+    ls[j & 7] += e0 + e1;
+    pk[j] = pack_bf16x2(e0, e1);
+  }
+  tmem_st16(tS + c * 16, pk);
 }
 
 }  // namespace
@@ -133,7 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_addr(&sm.s_full[i]), 1);
-      mbar_init(smem_addr(&sm.p_full[i]), 128);
+      mbar_init(smem_addr(&sm.p_full[i][0]), 128);
+      mbar_init(smem_addr(&sm.p_full[i][1]), 128);
       mbar_init(smem_addr(&sm.o_done[i]), 1);
     }
     mbar_init(smem_addr(&sm.drain), 1);
@@ -281,11 +299,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t nk_addr = smem_addr(&sm.kv[nst][0]);
           // Query tile 0: PV0(cur), then S0(next).
           if (entry_c0(cur) != kSkip) {
-            ok = mbar_wait(smem_addr(&sm.p_full[0]), p_cnt0 & 1, ctl);
+            // First half of P (keys 0-63), then the second half.
+            ok = mbar_wait(smem_addr(&sm.p_full[0][0]), p_cnt0 & 1, ctl);
             if (!ok) break;
-            ++p_cnt0;
             tc_fence_after();
-            issue_pv<D>(tO0, tS0, v_addr, acc0);
+            issue_pv<D, 0, 4>(tO0, tS0, v_addr, acc0);
+            ok = mbar_wait(smem_addr(&sm.p_full[0][1]), p_cnt0 & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv<D, 4, 8>(tO0, tS0, v_addr, true);
+            ++p_cnt0;
             acc0 = true;
             if (e == last0) umma_commit(smem_addr(&sm.o_done[0]));
           }
@@ -295,11 +318,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // Query tile 1: PV1(cur), then S1(next).
           if (entry_c1(cur) != kSkip) {
-            ok = mbar_wait(smem_addr(&sm.p_full[1]), p_cnt1 & 1, ctl);
+            // First half of P (keys 0-63), then the second half.
+            ok = mbar_wait(smem_addr(&sm.p_full[1][0]), p_cnt1 & 1, ctl);
             if (!ok) break;
-            ++p_cnt1;
             tc_fence_after();
-            issue_pv<D>(tO1, tS1, v_addr, acc1);
+            issue_pv<D, 0, 4>(tO1, tS1, v_addr, acc1);
+            ok = mbar_wait(smem_addr(&sm.p_full[1][1]), p_cnt1 & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv<D, 4, 8>(tO1, tS1, v_addr, true);
+            ++p_cnt1;
             acc1 = true;
             if (e == last1) umma_commit(smem_addr(&sm.o_done[1]));
           }
@@ -389,55 +417,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float m_use = m_run == -INFINITY ? 0.f : m_run;
         float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (cls == kMasked) {
-          // Masked tiles: every exponential on the MUFU unit, so -inf gives exactly 0.
+        const bool rescale_o = ntile > 0 && __any_sync(0xffffffffu, resc);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
+        for (int h = 0; h < 2; ++h) {
+          softmax_chunk(s, 2 * h, sl2, m_use, tS, ls);
+          softmax_chunk(s, 2 * h + 1, sl2, m_use, tS, ls);
+          if (h == 0) {
+            if (rescale_o) {
+              // O holds the previous PV products (complete: this tile's s_full was
+              // committed after them) and no PV of this tile starts before
+              // p_full: rescale it in place.
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float e0 = ex2_approx(fmaf(s[c * 32 + 2 * j], sl2, -m_use));
-              const float e1 = ex2_approx(fmaf(s[c * 32 + 2 * j + 1], sl2, -m_use));
-              ls[j & 7] += e0 + e1;
-              pk[j] = pack_bf16x2(e0, e1);
+              for (int c = 0; c < D; c += 32) {
+                uint32_t o[32];
+                tmem_ld32(tO + c, o);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+                tmem_st32(tO + c, o);
+              }
             }
-            tmem_st16(tS + c * 16, pk);
-          }
-        } else {
-          // Full tiles: one column pair in kPolyEvery takes its exponentials on the FMA pipe.
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float x0 = fmaf(s[c * 32 + 2 * j], sl2, -m_use);
-              const float x1 = fmaf(s[c * 32 + 2 * j + 1], sl2, -m_use);
-              const bool poly = kPolyEvery > 0 && (j % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
-              const float e0 = poly ? ex2_poly(x0) : ex2_approx(x0);
-              const float e1 = poly ? ex2_poly(x1) : ex2_approx(x1);
-              ls[j & 7] += e0 + e1;
-              pk[j] = pack_bf16x2(e0, e1);
-            }
-            tmem_st16(tS + c * 16, pk);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(smem_addr(&sm.p_full[wg][0]));
           }
         }
         const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-        if (ntile > 0 && __any_sync(0xffffffffu, resc)) {
-          // O holds the previous PV products (complete: this tile's s_full was
-          // committed after them) and the next PV waits for p_full: rescale in place.
-#pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(tO + c, o);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            tmem_st32(tO + c, o);
-          }
-        }
         l_run += lsum;
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(smem_addr(&sm.p_full[wg]));
+        mbar_arrive(smem_addr(&sm.p_full[wg][1]));
         ++ntile;
       }
       if (!ok) break;

@@ -280,16 +280,6 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Warpgroup register re-split (all four warps of a warpgroup execute the same one).
-template <int N>
-__device__ __forceinline__ void regs_increase() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void regs_decrease() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -304,22 +294,19 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
-// 2^x on the FMA/ALU pipes instead of the MUFU unit, for x <= 8.
-// Method: Cody-Waite style range reduction x = n + f, n = round(x) obtained by
-// adding 1.5 * 2^23 (the integer lands in the low mantissa bits, f in
-// [-1/2, 1/2]); 2^f by a degree-3 polynomial whose coefficients minimise the
-// maximum relative error on [-1/2, 1/2] (Remez exchange, fitted by
-// csrc/gen_exp2_poly.py: max relative error 7.5e-5); 2^n applied by adding n to
-// the exponent field. Inputs below -125 are clamped to -125 (result ~2^-125, not
-// 0): callers use it only where no -inf occurs.
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(5.517166853e-02f, f, 2.426111251e-01f), f, 6.932609677e-01f), f,
-                       9.999280572e-01f);
-  // (bits(t) << 23) == n << 23: the rounding constant's low 9 bits are zero.
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+// Packed fp32 pair arithmetic (sm_100 f32x2): two lanes per instruction.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
