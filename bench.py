@@ -51,6 +51,24 @@ def dist_env():
     return ws, rank, local
 
 
+def job_throughput(local_ms: float, flops_per_rank: float, world_size: int, device=None) -> tuple:
+    """Whole-job throughput of independent per-rank replicas (weak scaling).
+
+    Every rank ran the same work; the job time is the maximum of the ranks'
+    device-timed milliseconds (one all-reduce MAX when world_size > 1, on
+    whatever process group is initialised). Returns (job_ms, TFLOP/s over all
+    ranks).
+    """
+    job_ms = float(local_ms)
+    if world_size > 1:
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([job_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        job_ms = float(t.item())
+    return job_ms, world_size * flops_per_rank / (job_ms * 1e-3) / 1e12
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle samples while the timed region runs."""
 
@@ -69,7 +87,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
         time.sleep(0.3)
@@ -135,7 +153,7 @@ def run_reference(args):
         return 0
     from workloads import WORKLOADS
     w = WORKLOADS[WORKLOAD]
-    per_step = 12.0
+    per_step = 5.0
     rates, secs = [], []
     for i in range(args.warmup + args.steps):
         tf, rows, dt, cores = oracle_sample_rate(w, max_rows=4096, budget_s=per_step)
@@ -161,12 +179,12 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", action="store_true",
-                    help="only launch the fused attention kernel warmup+steps times (for ncu captures)")
+    ap.add_argument("--profile", choices=["attn", "merge", "permute"], default=None,
+                    help="only launch one kernel warmup+steps times (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -210,20 +228,25 @@ def main():
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    def max_over_ranks(x: float) -> float:
-        if ws == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     if args.profile:
         for x, y in ((q, qz), (k, kz), (v, vz)):
             cp.layout_permute(plan, x, 0, out=y)
+        if args.profile == "merge":
+            op = torch.empty(N, plan.rows, D, dtype=torch.float32, device=dev)
+            lp = torch.empty(N, plan.rows, dtype=torch.float32, device=dev)
+            cp.attn_fwd_partials(plan, qz, kz, vz, o_parts=op, lse_parts=lp)
+            om = torch.empty(plan.rows, D, dtype=torch.bfloat16, device=dev)
+            lm = torch.empty(plan.rows, dtype=torch.float32, device=dev)
         for _ in range(args.warmup + args.steps):
-            cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=lse)
+            if args.profile == "attn":
+                cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=lse)
+            elif args.profile == "merge":
+                cp.merge_partials(op, lp, o_out=om, lse_out=lm)
+            else:
+                cp.layout_permute(plan, q, 0, out=qz)
         st = cp.check(plan)
-        print(json.dumps({"profile": "attn_fwd", "launches": args.warmup + args.steps, "status": st}))
+        print(json.dumps({"profile": args.profile, "launches": args.warmup + args.steps, "status": st}))
         return 0 if st == 0 else 1
 
     for _ in range(args.warmup):
@@ -243,8 +266,7 @@ def main():
     st = cp.check(plan)
     if st != 0:
         raise RuntimeError(f"timed run failed: {cp.status_string(st)}")
-    ms = max_over_ranks(ev0.elapsed_time(ev1)) / args.steps
-    value = ws * w.flops / (ms * 1e-3) / 1e12
+    ms, value = job_throughput(ev0.elapsed_time(ev1) / args.steps, w.flops, ws, dev)
 
     # --- attention kernel alone (dominant kernel), CUDA events on its stream
     att_ms = []
@@ -315,8 +337,7 @@ def main():
         e2e_step()
     e1.record(stream)
     barrier()
-    e_ms = max_over_ranks(e0.elapsed_time(e1)) / e_steps
-    e2e_value = ws * w.flops / (e_ms * 1e-3) / 1e12
+    e_ms, e2e_value = job_throughput(e0.elapsed_time(e1) / e_steps, w.flops, ws, dev)
     h2d = 3 * q.numel() * 2
     d2h = o.numel() * 2 + lse.numel() * 4
 
