@@ -30,6 +30,7 @@ SIGNATURES = {
     "cp_attn_plan_destroy": (_I, [_P]),
     "cp_attn_plan_tile_counts": (_I64, [_P, _P]),
     "cp_attn_plan_num_items": (_I64, [_P]),
+    "cp_attn_plan_cta_loads": (_I64, [_P, _P]),
     "cp_attn_workspace_bytes": (_SZ, [_P, _I]),
     "cp_attn_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "cp_attn_fwd_partials": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
@@ -125,6 +126,15 @@ class Plan:
 
     def num_items(self) -> int:
         return int(lib().cp_attn_plan_num_items(self._h))
+
+    def cta_loads(self):
+        """Modelled load of each CTA of the kernel's static schedule."""
+        n = int(lib().cp_attn_plan_cta_loads(self._h, None))
+        if n < 0:
+            raise CpAttnError("cp_attn_plan_cta_loads", n)
+        arr = (ctypes.c_int64 * max(n, 1))()
+        lib().cp_attn_plan_cta_loads(self._h, ctypes.cast(arr, ctypes.c_void_p))
+        return list(arr)[:n]
 
     def workspace_bytes(self, with_partials: bool = False) -> int:
         return int(lib().cp_attn_workspace_bytes(self._h, int(with_partials)))

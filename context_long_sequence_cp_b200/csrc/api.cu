@@ -9,6 +9,8 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <queue>
+#include <utility>
 #include <vector>
 
 #include "attn_fwd.h"
@@ -35,11 +37,17 @@ struct cp_attn_plan_s {
   std::vector<uint32_t> entries;
   int* d_step_off = nullptr;
   uint32_t* d_entries = nullptr;
+  // Static schedule: CTA c runs items [cta_begin[c], cta_begin[c+1]) in order.
+  int n_cta = 0;
+  std::vector<int> cta_begin;
+  std::vector<int64_t> cta_load;    // modelled cost per CTA (key tiles + item overhead)
+  int* d_cta_begin = nullptr;
 };
 
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per in-kernel wait
+constexpr int kDefaultSmCount = 148;               // B200; used when no device is visible
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -89,6 +97,51 @@ void item_cost(const Geometry& g, int rq, int qp, int t0, int t1, int* c0n, int*
   }
 }
 
+// Modelled cost of an item in executed key tiles: the tiles of its walk plus a
+// fixed overhead for loading its query tiles, the first score product and the
+// output write, measured at about one and a half key tiles.
+constexpr int64_t kItemOverheadHalfTiles = 3;
+
+// Assigns the sorted work list to n_cta persistent CTAs: each item, in list
+// order, goes to the CTA whose modelled finish time is the earliest (ties to the
+// lower index). Items therefore start in about list order (so that the items
+// running together still share keys and values in L2) while the CTAs finish
+// together. The list is reordered so that each CTA's items are contiguous.
+void schedule_items(cp_attn_plan_s* p, int n_cta) {
+  const int n = static_cast<int>(p->items.size());
+  std::vector<int64_t> cost(n);
+  for (int i = 0; i < n; ++i) {
+    const WorkItem& w = p->items[i];
+    const int rq = w.rb / p->g.B;
+    const int* off = p->step_off.data() + static_cast<size_t>(rq * p->npairs + w.qp) * (p->g.NR + 1);
+    cost[i] = 2 * static_cast<int64_t>(off[p->g.NR] - off[0]) + kItemOverheadHalfTiles;
+  }
+  n_cta = n < n_cta ? n : n_cta;
+  p->n_cta = n_cta;
+  p->cta_load.assign(n_cta, 0);
+  std::vector<int> owner(n);
+  using Slot = std::pair<int64_t, int>;
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> free_at;
+  for (int c = 0; c < n_cta; ++c) free_at.push(Slot(0, c));
+  for (int i = 0; i < n; ++i) {
+    const Slot s = free_at.top();
+    free_at.pop();
+    owner[i] = s.second;
+    p->cta_load[s.second] = s.first + cost[i];
+    free_at.push(Slot(s.first + cost[i], s.second));
+  }
+  std::vector<WorkItem> sorted;
+  sorted.reserve(n);
+  p->cta_begin.assign(n_cta + 1, 0);
+  for (int c = 0; c < n_cta; ++c) {
+    p->cta_begin[c] = static_cast<int>(sorted.size());
+    for (int i = 0; i < n; ++i)
+      if (owner[i] == c) sorted.push_back(p->items[i]);
+  }
+  p->cta_begin[n_cta] = n;
+  p->items.swap(sorted);
+}
+
 int ensure_device(cp_attn_plan_s* p) {
   if (p->d_items != nullptr) return CP_OK;
   return CP_ERR_CUDA;
@@ -109,6 +162,8 @@ int launch_view(cp_attn_plan_s* p, const Geometry& g, const void* q, const void*
   P.scale_log2 = p->scale * 1.4426950408889634f;
   P.items = p->d_items;
   P.n_items = static_cast<int>(p->items.size());
+  P.cta_begin = p->d_cta_begin;
+  P.n_cta = p->n_cta;
   P.step_off = p->d_step_off;
   P.entries = p->d_entries;
   P.npairs = p->npairs;
@@ -220,23 +275,35 @@ int cp_attn_plan(cp_attn_plan_t* out, int B, int H, int S, int D, int N, int cau
       }
     }
   }
-  // Items that read the same keys/values (same batch and head) are kept together
-  // so that the ones running at the same time share them in L2; within a group
-  // the most expensive come first.
+  // Items that read the same keys/values (same batch, heads in pairs) are kept
+  // together so that the ones running at the same time share them in L2; within
+  // a group the most expensive come first. Pairs of heads (rather than single
+  // heads) give the schedule below enough large items late in the list to end
+  // level (modelled max/mean CTA load 1.005 instead of 1.024 on 32 heads).
   std::stable_sort(p->items.begin(), p->items.end(), [&](const WorkItem& a, const WorkItem& b) {
     const int ba = a.rb % g.B, bb = b.rb % g.B;
     if (ba != bb) return ba < bb;
-    if (a.h != b.h) return a.h < b.h;
+    if (a.h / 2 != b.h / 2) return a.h / 2 < b.h / 2;
     return a.cost > b.cost;
   });
 
   int ndev = 0;
-  if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0) {
+  const bool have_device = cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0;
+  int sms = kDefaultSmCount;
+  if (have_device) {
     cudaGetDevice(&p->device);
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess || sms <= 0)
+      sms = kDefaultSmCount;
+  }
+  schedule_items(p, sms);
+  if (have_device) {
     const size_t bytes = p->items.size() * sizeof(WorkItem);
     const size_t off_bytes = p->step_off.size() * sizeof(int);
     const size_t ent_bytes = p->entries.size() * sizeof(uint32_t);
+    const size_t cta_bytes = p->cta_begin.size() * sizeof(int);
     bool ok = cudaMalloc(&p->d_items, bytes > 0 ? bytes : sizeof(WorkItem)) == cudaSuccess &&
+              cudaMalloc(&p->d_cta_begin, cta_bytes) == cudaSuccess &&
+              cudaMemcpy(p->d_cta_begin, p->cta_begin.data(), cta_bytes, cudaMemcpyHostToDevice) == cudaSuccess &&
               cudaMalloc(&p->d_status, sizeof(int)) == cudaSuccess &&
               cudaMalloc(&p->d_step_off, off_bytes) == cudaSuccess &&
               cudaMalloc(&p->d_entries, ent_bytes > 0 ? ent_bytes : sizeof(uint32_t)) == cudaSuccess &&
@@ -247,6 +314,8 @@ int cp_attn_plan(cp_attn_plan_t* out, int B, int H, int S, int D, int N, int cau
               cudaMemset(p->d_status, 0, sizeof(int)) == cudaSuccess;
     if (!ok) {
       cudaFree(p->d_items);
+      cudaFree(p->d_cta_begin);
+      p->d_cta_begin = nullptr;
       cudaFree(p->d_status);
       cudaFree(p->d_step_off);
       cudaFree(p->d_entries);
@@ -265,6 +334,7 @@ int cp_attn_plan(cp_attn_plan_t* out, int B, int H, int S, int D, int N, int cau
 int cp_attn_plan_destroy(cp_attn_plan_t plan) {
   if (plan == nullptr) return CP_OK;
   if (plan->d_items != nullptr) cudaFree(plan->d_items);
+  if (plan->d_cta_begin != nullptr) cudaFree(plan->d_cta_begin);
   if (plan->d_status != nullptr) cudaFree(plan->d_status);
   if (plan->d_step_off != nullptr) cudaFree(plan->d_step_off);
   if (plan->d_entries != nullptr) cudaFree(plan->d_entries);
@@ -285,6 +355,13 @@ int64_t cp_attn_plan_tile_counts(cp_attn_plan_t plan, int64_t* per_rank) {
 int64_t cp_attn_plan_num_items(cp_attn_plan_t plan) {
   if (plan == nullptr) return CP_ERR_INVALID_ARG;
   return static_cast<int64_t>(plan->items.size());
+}
+
+int64_t cp_attn_plan_cta_loads(cp_attn_plan_t plan, int64_t* per_cta) {
+  if (plan == nullptr) return CP_ERR_INVALID_ARG;
+  if (per_cta != nullptr)
+    for (int c = 0; c < plan->n_cta; ++c) per_cta[c] = plan->cta_load[c];
+  return plan->n_cta;
 }
 
 size_t cp_attn_workspace_bytes(cp_attn_plan_t plan, int with_partials) {

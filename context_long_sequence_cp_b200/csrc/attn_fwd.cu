@@ -76,8 +76,18 @@ struct alignas(1024) Smem {
   uint64_t o_done[2];
   uint64_t drain;
   uint32_t tmem_base;
-  int abort;
+  WaitBlock wblk;
 };
+
+// Loads a work item with a volatile access, which the compiler cannot merge with
+// an earlier load of the same item.
+__device__ __forceinline__ WorkItem ld_item_volatile(const WorkItem* ptr) {
+  int4 v;
+  asm volatile("ld.global.nc.v4.s32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(ptr));
+  return WorkItem{v.x, v.y, v.z, v.w};
+}
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
@@ -155,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_addr(&sm.o_done[i]), 1);
     }
     mbar_init(smem_addr(&sm.drain), 1);
-    sm.abort = 0;
+    wait_block_init(sm.wblk, p.status, p.wait_limit_ns);
     fence_barrier_init();
   }
   if (warp == 8) {
@@ -171,7 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
-  WaitCtl ctl{&sm.abort, p.status, p.wait_limit_ns};
+  const WaitCtl ctl = wait_ctl(sm.wblk);
+  const int it_end = __ldg(p.cta_begin + blockIdx.x + 1);   // this CTA's items end here
 
   // Every role walks the same precomputed key list of each work item.
   const int nstep_off = g.NR + 1;
@@ -184,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int q_iter = 0;
       int kv_idx = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
+      for (int it = __ldg(p.cta_begin + blockIdx.x); it < it_end && ok; ++it) {
         const WorkItem w = p.items[it];
         const int rq = w.rb / g.B;
         const int bv = w.rb - rq * g.B;
@@ -237,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int q_iter = 0, kv_idx = 0;
       int p_cnt0 = 0, p_cnt1 = 0;
       bool ok = true, issued = false;
-      for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
+      for (int it = __ldg(p.cta_begin + blockIdx.x); it < it_end && ok; ++it) {
         const WorkItem w = p.items[it];
         const int rq = w.rb / g.B;
         const int* off = p.step_off + (rq * p.npairs + w.qp) * nstep_off;
@@ -361,16 +372,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cls_shift = wg == 0 ? 25 : 27;
     int s_cnt = 0, od_cnt = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
-      const WorkItem w = p.items[it];
-      const int rq = w.rb / g.B;
-      const int bv = w.rb - rq * g.B;
-      const int q_first = w.qp * kPair;
-      const int tl = q_first + wg * kTile + row;
-      const bool valid = tl < g.T;
-      const int64_t gq = global_pos(g, rq, valid ? tl : g.T - 1);
-      const int* off = p.step_off + (rq * p.npairs + w.qp) * nstep_off;
-      const int e_begin = __ldg(off + p.t_begin), e_end = __ldg(off + p.t_end);
+    for (int it = __ldg(p.cta_begin + blockIdx.x); it < it_end && ok; ++it) {
+      int64_t gq;
+      bool valid;
+      int e_begin, e_end;
+      {
+        const WorkItem w = p.items[it];
+        const int rq = w.rb / g.B;
+        const int tl = w.qp * kPair + wg * kTile + row;
+        valid = tl < g.T;
+        gq = global_pos(g, rq, valid ? tl : g.T - 1);
+        const int* off = p.step_off + (rq * p.npairs + w.qp) * nstep_off;
+        e_begin = __ldg(off + p.t_begin);
+        e_end = __ldg(off + p.t_end);
+      }
       float m_run = -INFINITY, l_run = 0.f;
       int ntile = 0;
       uint32_t ent = e_begin < e_end ? __ldg(p.entries + e_begin) : 0u;
@@ -428,12 +443,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               // committed after them) and no PV of this tile starts before
               // p_full: rescale it in place.
 #pragma unroll
-              for (int c = 0; c < D; c += 32) {
-                uint32_t o[32];
-                tmem_ld32(tO + c, o);
+              for (int c = 0; c < D; c += 16) {
+                uint32_t o[16];
+                tmem_ld16(tO + c, o);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-                tmem_st32(tO + c, o);
+                for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+                tmem_st16(tO + c, o);
               }
             }
             tmem_st_wait();
@@ -450,6 +465,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
+      // The item's fields again: a fresh load, so that they are not kept live
+      // across the key loop in registers the scores need.
+      const WorkItem w = ld_item_volatile(p.items + it);
+      const int bv = w.rb % g.B;
+      const int tl = w.qp * kPair + wg * kTile + row;
       const int64_t row_id = (static_cast<int64_t>(w.rb) * g.T + tl) * g.Hh + w.h;
       if (ntile > 0) {
         ok = mbar_wait(smem_addr(&sm.o_done[wg]), od_cnt & 1, ctl);
@@ -532,12 +552,7 @@ cudaError_t launch_impl(const FwdLaunch& L, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0;
-  e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  const int grid = L.params.n_items < sms ? L.params.n_items : sms;
+  const int grid = L.params.n_cta;   // the schedule's CTA count (normally the SM count)
   if (grid <= 0) return cudaSuccess;
   kern<<<grid, kThreads, smem, stream>>>(L.tm_q, L.tm_k, L.tm_v, L.params);
   return cudaGetLastError();

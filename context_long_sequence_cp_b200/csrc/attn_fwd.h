@@ -17,6 +17,8 @@ struct FwdParams {
   float scale_log2;            // softmax scale * log2(e)
   const WorkItem* items;       // device work list
   int n_items;
+  const int* cta_begin;        // CTA c runs items [cta_begin[c], cta_begin[c+1])
+  int n_cta;                   // grid size the schedule was made for
   // Precomputed key walks: the walk of query-tile pair (rq, qp) over ring step t
   // is entries[step_off[(rq*npairs + qp)*(NR+1) + t] .. step_off[... + t + 1]).
   const int* step_off;

@@ -165,12 +165,11 @@ __global__ void index_map_kernel(UnitMap m, int64_t units, int64_t* __restrict__
 // barrier that nothing arrives on; the wait runs out and records the timeout.
 __global__ void wait_probe_kernel(int* status, uint64_t limit_ns) {
   __shared__ uint64_t bar;
-  __shared__ int abort_flag;
+  __shared__ sm100::WaitBlock wblk;
   if (threadIdx.x == 0) {
     sm100::mbar_init(sm100::smem_addr(&bar), 1);
-    abort_flag = 0;
+    const sm100::WaitCtl ctl = sm100::wait_block_init(wblk, status, limit_ns);
     sm100::fence_barrier_init();
-    sm100::WaitCtl ctl{&abort_flag, status, limit_ns};
     sm100::mbar_wait(sm100::smem_addr(&bar), 0, ctl);
   }
 }

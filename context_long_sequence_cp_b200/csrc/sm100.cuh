@@ -60,29 +60,52 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Status codes shared with the host (values of the public CP_ERR_* enum).
 constexpr int kStatusTimeout = -5;
 
-struct WaitCtl {
-  volatile int* abort;     // CTA-wide flag in shared memory
-  int* status;             // global status word of the plan
-  uint64_t limit_ns;       // budget of one wait
+// State of the bounded waits of one CTA, kept in shared memory so that a wait
+// call carries one 32-bit address instead of pointers and limits in registers.
+struct WaitBlock {
+  int* status;                  // global status word of the plan
+  unsigned long long limit_ns;  // budget of one wait
+  int abort;                    // CTA-wide abort flag
+  int pad;
 };
 
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, WaitCtl ctl) {
+// Shared-memory address of a WaitBlock.
+struct WaitCtl {
+  uint32_t wb;
+};
+
+__device__ __forceinline__ WaitCtl wait_block_init(WaitBlock& b, int* status, unsigned long long limit_ns) {
+  b.status = status;
+  b.limit_ns = limit_ns;
+  b.abort = 0;
+  return WaitCtl{smem_addr(&b)};
+}
+
+__device__ __forceinline__ WaitCtl wait_ctl(const WaitBlock& b) { return WaitCtl{smem_addr(&b)}; }
+
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint32_t wb) {
   const uint64_t t0 = globaltimer_ns();
+  uint64_t limit;
+  asm volatile("ld.shared.u64 %0, [%1];" : "=l"(limit) : "r"(wb + 8));
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*ctl.abort) return false;
-    if (globaltimer_ns() - t0 > ctl.limit_ns) {
-      *ctl.abort = 1;
-      atomicCAS(ctl.status, 0, kStatusTimeout);
+    int ab;
+    asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(ab) : "r"(wb + 16));
+    if (ab) return false;
+    if (globaltimer_ns() - t0 > limit) {
+      asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(wb + 16), "r"(1) : "memory");
+      uint64_t st;
+      asm volatile("ld.shared.u64 %0, [%1];" : "=l"(st) : "r"(wb));
+      atomicCAS(reinterpret_cast<int*>(st), 0, kStatusTimeout);
       return false;
     }
   }
 }
 
 // Wait for the phase with the given parity to complete; false on abort/timeout.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, WaitCtl ctl) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, ctl);
+  return mbar_wait_slow(bar, parity, ctl.wb);
 }
 
 // Drain wait used on the abort path: ignores the abort flag, own budget.
@@ -217,6 +240,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 
 // Two back-to-back 32-column loads with a single wait (more loads in flight).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[32], uint32_t (&s)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "

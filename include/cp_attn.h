@@ -116,6 +116,17 @@ CP_API int64_t cp_attn_plan_tile_counts(cp_attn_plan_t plan, int64_t* per_rank);
 CP_API int64_t cp_attn_plan_num_items(cp_attn_plan_t plan);
 
 /*
+ * Static schedule of the attention kernel: one persistent CTA per SM runs a
+ * contiguous run of the work list, assigned at plan time by giving each item,
+ * in list order, to the CTA with the earliest modelled finish. The model counts
+ * two units per executed key tile of the item plus three per item. Writes each
+ * CTA's modelled load to per_cta[n_cta] (host memory, may be NULL) and returns
+ * n_cta (the SM count of the device current at plan time, 148 when none is
+ * visible, capped by the number of items), or a negative status.
+ */
+CP_API int64_t cp_attn_plan_cta_loads(cp_attn_plan_t plan, int64_t* per_cta);
+
+/*
  * Workspace bytes needed by cp_attn_fwd (with_partials = 0) or
  * cp_attn_fwd_partials (with_partials = 1). 0 for contiguous/zigzag fused
  * calls; 4 * B*S*H*D*2 bytes (Q, K, V and O head groups) for Ulysses.

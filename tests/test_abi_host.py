@@ -9,6 +9,7 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
 
 import context_long_sequence_cp_b200 as cp
@@ -114,3 +115,44 @@ def test_workspace_and_map_sizes():
     assert z.workspace_bytes(False) == 0 and z.workspace_bytes(True) == 0
     assert z.index_map_len() == 4096
     assert z.num_items() == 4 * 16 * 4     # ranks x heads x query-tile pairs (T=1024)
+
+
+def _executed_key_tiles(S, N, layout, causal, tile=128):
+    """Key tiles walked per (batch, head): a key tile counts once per query-tile
+    pair in which at least one of the two query tiles has an allowed key in it."""
+    from oracle.layouts import chunk_positions
+    pos = chunk_positions(S, N, layout)
+    T = S // N
+    nt = -(-T // tile)
+    tmin = np.array([[pos[r, i * tile:(i + 1) * tile].min() for i in range(nt)] for r in range(N)])
+    tmax = np.array([[pos[r, i * tile:(i + 1) * tile].max() for i in range(nt)] for r in range(N)])
+    total = 0
+    for r in range(N):
+        for t in range(N):
+            rk = (r + t) % N
+            ok = tmin[rk][None, :] <= tmax[r][:, None] if causal else np.ones((nt, nt), bool)
+            for qp in range(-(-nt // 2)):
+                rows = ok[2 * qp:2 * qp + 2]
+                total += int(rows.any(axis=0).sum())
+    return total
+
+
+@pytest.mark.parametrize("layout", ["zigzag", "contiguous"])
+def test_static_schedule_is_balanced_and_complete(layout):
+    w = WORKLOADS["zigzag_32k"]
+    p = cp.Plan(w.B, w.H, w.S, w.D, w.N, True, layout)
+    loads = np.array(p.cta_loads())
+    assert len(loads) == 148                        # one CTA per SM (no device here: 148)
+    assert loads.max() / loads.mean() < 1.02
+    # Modelled load = 2 per walked key tile + 3 per item, so the loads add up to
+    # the work of every item exactly once.
+    walked = _executed_key_tiles(w.S, w.N, layout, True) * w.H
+    assert loads.sum() == 2 * walked + 3 * p.num_items()
+
+
+def test_static_schedule_small_plan_one_item_per_cta():
+    p = cp.Plan(1, 2, 256, 64, 4, False, "contiguous")   # 4 ranks x 2 heads x 1 pair
+    loads = p.cta_loads()
+    assert len(loads) == p.num_items() == 8
+    # Non-causal: every item walks all 4 ranks' single key tile.
+    assert loads == [2 * 4 + 3] * 8
