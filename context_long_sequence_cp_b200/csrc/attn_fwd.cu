@@ -99,7 +99,7 @@ __device__ __forceinline__ void issue_s(uint32_t tS, uint32_t q_addr, uint32_t k
     const uint32_t off = (kk >> 2) * Cfg<D>::kBlockBytes + (kk & 3) * 32;
     const uint64_t a = smem_desc_sw128(q_addr + off, 16, 1024);
     const uint64_t b = smem_desc_sw128(k_addr + off, 16, 1024);
-    umma_ss(tS, a, b, Cfg<D>::kIdescS, kk > 0 ? 1u : 0u);
+    umma_ss_elect(tS, a, b, Cfg<D>::kIdescS, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -111,7 +111,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint32_t v_ad
 #pragma unroll
   for (int kk = KK_BEGIN; kk < KK_END; ++kk) {
     const uint64_t b = smem_desc_sw128(v_addr + kk * 2048, Cfg<D>::kBlockBytes, 1024);
-    umma_ts(tO, tP + kk * 8, b, Cfg<D>::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+    umma_ts_elect(tO, tP + kk * 8, b, Cfg<D>::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -134,6 +134,36 @@ __device__ __forceinline__ void softmax_chunk(const float (&s)[kTile], int c, fl
     pk[j] = pack_bf16x2(e0, e1);
   }
   tmem_st16(tS + c * 16, pk);
+}
+
+// Maximum of the 64 scores s[32c .. 32c+63], four chains of 3-input maxima.
+__device__ __forceinline__ float half_max(const float (&s)[kTile], int c) {
+  float m[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int b = 32 * c + 16 * k;
+    float x = max3(s[b], s[b + 1], s[b + 2]);
+#pragma unroll
+    for (int j = 3; j + 1 < 16; j += 2) x = max3(x, s[b + j], s[b + j + 1]);
+    m[k] = fmaxf(x, s[b + 15]);
+  }
+  return fmaxf(max3(m[0], m[1], m[2]), m[3]);
+}
+
+// Multiplies the 64 bf16 P values of keys 0-63 (TMEM columns tS .. tS+31, two
+// per column) by beta.
+__device__ __forceinline__ void rescale_p_half(uint32_t tS, float beta) {
+#pragma unroll
+  for (int c = 0; c < 32; c += 16) {
+    uint32_t v[16];
+    tmem_ld16(tS + c, v);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&v[q]);
+      v[q] = pack_bf16x2(__low2float(b) * beta, __high2float(b) * beta);
+    }
+    tmem_st16(tS + c, v);
+  }
 }
 
 }  // namespace
@@ -189,7 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 9) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane issues each load.
+    {
       const uint64_t pol_q = l2_policy_evict_first();
       const uint64_t pol_kv = l2_policy_evict_last();
       int q_iter = 0;
@@ -203,12 +234,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int* off = p.step_off + (rq * p.npairs + w.qp) * nstep_off;
         const int e_begin = __ldg(off + p.t_begin), e_end = __ldg(off + p.t_end);
         if (q_iter > 0) ok = mbar_wait(smem_addr(&sm.q_empty), (q_iter - 1) & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         const uint32_t qbar = smem_addr(&sm.q_full);
-        mbar_arrive_expect_tx(qbar, 2 * C::kTileBytes);
+        mbar_arrive_expect_tx_elect(qbar, 2 * C::kTileBytes);
         for (int i = 0; i < 2; ++i)
           for (int blk = 0; blk < C::kBlocks; ++blk)
-            tma_load_4d(smem_addr(&sm.q[i][0]) + blk * C::kBlockBytes, &tm_q, qbar, blk * 64, w.h,
+            tma_load_4d_elect(smem_addr(&sm.q[i][0]) + blk * C::kBlockBytes, &tm_q, qbar, blk * 64, w.h,
                         q0 + i * kTile, w.rb, pol_q);
         ++q_iter;
         for (int e = e_begin; e < e_end && ok; ++e) {
@@ -219,12 +251,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int stage = kv_idx % C::kStages;
             const int round = kv_idx / C::kStages;
             if (round > 0) ok = mbar_wait(smem_addr(&sm.kv_empty[stage]), (round - 1) & 1, ctl);
+            ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             const uint32_t bar = smem_addr(&sm.kv_full[stage]);
-            mbar_arrive_expect_tx(bar, C::kTileBytes);
+            mbar_arrive_expect_tx_elect(bar, C::kTileBytes);
             const CUtensorMap* map = which == 0 ? &tm_k : &tm_v;
             for (int blk = 0; blk < C::kBlocks; ++blk)
-              tma_load_4d(smem_addr(&sm.kv[stage][0]) + blk * C::kBlockBytes, map, bar, blk * 64, w.h, k0,
+              tma_load_4d_elect(smem_addr(&sm.kv[stage][0]) + blk * C::kBlockBytes, map, bar, blk * 64, w.h, k0,
                           rbk, pol_kv);
             ++kv_idx;
           }
@@ -241,7 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane issues each MMA and commit.
+    {
       const uint32_t tS0 = tbase, tS1 = tbase + 128;
       const uint32_t tO0 = tbase + C::kOCol, tO1 = tbase + C::kOCol + D;
       const uint32_t q_addr0 = smem_addr(&sm.q[0][0]), q_addr1 = smem_addr(&sm.q[1][0]);
@@ -261,17 +295,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (entry_c1(ent) != kSkip) last1 = e;
         }
         ok = mbar_wait(smem_addr(&sm.q_full), q_iter & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++q_iter;
         tc_fence_after();
         if (e_begin == e_end) {
-          umma_commit(smem_addr(&sm.q_empty));
+          umma_commit_elect(smem_addr(&sm.q_empty));
           continue;
         }
         // First key tile: its S products.
         uint32_t cur = __ldg(p.entries + e_begin);
         int kst = kv_idx % C::kStages;
         ok = mbar_wait(smem_addr(&sm.kv_full[kst]), (kv_idx / C::kStages) & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++kv_idx;
         tc_fence_after();
@@ -279,15 +315,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t k_addr = smem_addr(&sm.kv[kst][0]);
           if (entry_c0(cur) != kSkip) {
             issue_s<D>(tS0, q_addr0, k_addr);
-            umma_commit(smem_addr(&sm.s_full[0]));
+            umma_commit_elect(smem_addr(&sm.s_full[0]));
           }
           if (entry_c1(cur) != kSkip) {
             issue_s<D>(tS1, q_addr1, k_addr);
-            umma_commit(smem_addr(&sm.s_full[1]));
+            umma_commit_elect(smem_addr(&sm.s_full[1]));
           }
         }
         issued = true;
-        umma_commit(smem_addr(&sm.kv_empty[kst]));
+        umma_commit_elect(smem_addr(&sm.kv_empty[kst]));
         bool acc0 = false, acc1 = false;
         for (int e = e_begin; e < e_end; ++e) {
           const bool has_next = e + 1 < e_end;
@@ -296,12 +332,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           // so that once P is ready the PV and the next S issue back to back.
           const int vst = kv_idx % C::kStages;
           ok = mbar_wait(smem_addr(&sm.kv_full[vst]), (kv_idx / C::kStages) & 1, ctl);
+          ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           ++kv_idx;
           int nst = 0;
           if (has_next) {
             nst = kv_idx % C::kStages;
             ok = mbar_wait(smem_addr(&sm.kv_full[nst]), (kv_idx / C::kStages) & 1, ctl);
+            ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             ++kv_idx;
           }
@@ -312,51 +350,55 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (entry_c0(cur) != kSkip) {
             // First half of P (keys 0-63), then the second half.
             ok = mbar_wait(smem_addr(&sm.p_full[0][0]), p_cnt0 & 1, ctl);
+            ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
             issue_pv<D, 0, 4>(tO0, tS0, v_addr, acc0);
             ok = mbar_wait(smem_addr(&sm.p_full[0][1]), p_cnt0 & 1, ctl);
+            ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
             issue_pv<D, 4, 8>(tO0, tS0, v_addr, true);
             ++p_cnt0;
             acc0 = true;
-            if (e == last0) umma_commit(smem_addr(&sm.o_done[0]));
+            if (e == last0) umma_commit_elect(smem_addr(&sm.o_done[0]));
           }
           if (has_next && entry_c0(nxt) != kSkip) {
             issue_s<D>(tS0, q_addr0, nk_addr);
-            umma_commit(smem_addr(&sm.s_full[0]));
+            umma_commit_elect(smem_addr(&sm.s_full[0]));
           }
           // Query tile 1: PV1(cur), then S1(next).
           if (entry_c1(cur) != kSkip) {
             // First half of P (keys 0-63), then the second half.
             ok = mbar_wait(smem_addr(&sm.p_full[1][0]), p_cnt1 & 1, ctl);
+            ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
             issue_pv<D, 0, 4>(tO1, tS1, v_addr, acc1);
             ok = mbar_wait(smem_addr(&sm.p_full[1][1]), p_cnt1 & 1, ctl);
+            ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
             issue_pv<D, 4, 8>(tO1, tS1, v_addr, true);
             ++p_cnt1;
             acc1 = true;
-            if (e == last1) umma_commit(smem_addr(&sm.o_done[1]));
+            if (e == last1) umma_commit_elect(smem_addr(&sm.o_done[1]));
           }
           if (has_next && entry_c1(nxt) != kSkip) {
             issue_s<D>(tS1, q_addr1, nk_addr);
-            umma_commit(smem_addr(&sm.s_full[1]));
+            umma_commit_elect(smem_addr(&sm.s_full[1]));
           }
-          if (has_next) umma_commit(smem_addr(&sm.kv_empty[nst]));
-          umma_commit(smem_addr(&sm.kv_empty[vst]));
+          if (has_next) umma_commit_elect(smem_addr(&sm.kv_empty[nst]));
+          umma_commit_elect(smem_addr(&sm.kv_empty[vst]));
           cur = nxt;
         }
         if (!ok) break;
-        umma_commit(smem_addr(&sm.q_empty));
+        umma_commit_elect(smem_addr(&sm.q_empty));
       }
       if (issued) {
         // Every tensor-core op (and the arrivals of its commits) must finish before
         // TMEM is freed and the CTA exits; on the abort path too.
-        umma_commit(smem_addr(&sm.drain));
+        umma_commit_elect(smem_addr(&sm.drain));
         mbar_wait_drain(smem_addr(&sm.drain), 0, p.wait_limit_ns);
       }
     }
@@ -408,54 +450,59 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < kTile; ++j) s[j] = j < lim ? s[j] : -INFINITY;
         }
-        // Row max: four independent chains of 3-input maxima (short dependency chains).
-        float mx;
-        {
-          float mc[4];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float m = s[32 * c];
-#pragma unroll
-            for (int j = 1; j + 1 < 32; j += 2) m = max3(m, s[32 * c + j], s[32 * c + j + 1]);
-            mc[c] = fmaxf(m, s[32 * c + 31]);
-          }
-          mx = fmaxf(max3(mc[0], mc[1], mc[2]), mc[3]);
-        }
-        const float m_tile = mx * sl2;
-        const float m_new = fmaxf(m_run, m_tile);
-        const bool resc = m_new - m_run > kRescaleThreshold;   // false while both are -inf
-        float alpha = 1.f;
-        if (resc) {
-          alpha = ex2_approx(m_run - m_new);   // 0 when m_run = -inf
-          m_run = m_new;
-          l_run *= alpha;
-        }
-        const float m_use = m_run == -INFINITY ? 0.f : m_run;
+        // Row max, then exponentials. The max of keys 0-63 comes first and their
+        // exponentials start at once; the max of keys 64-127 is computed while
+        // they run. Rescaling is lazy (only when the max grows by more than 2^8),
+        // so keys 64-127 rarely move the max; when they do, the stored P of keys
+        // 0-63 and its partial sums are scaled down to the new max before the
+        // MMA warp may read them.
+        const float m_prev = m_run;
+        float m01 = half_max(s, 0);
+        bool resc = m01 * sl2 - m_run > kRescaleThreshold;   // false while both are -inf
+        if (resc) m_run = m01 * sl2;
+        float m_use = m_run == -INFINITY ? 0.f : m_run;
         float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        const bool rescale_o = ntile > 0 && __any_sync(0xffffffffu, resc);
+        softmax_chunk(s, 0, sl2, m_use, tS, ls);
+        softmax_chunk(s, 1, sl2, m_use, tS, ls);
+        const float m23 = half_max(s, 2);
+        const bool resc_b = m23 * sl2 - m_run > kRescaleThreshold;
+        if (__any_sync(0xffffffffu, resc_b)) {
+          // Rare: keys 64-127 raise the max. P of keys 0-63 (32 packed columns)
+          // is scaled by 2^(m_use - m_use_new), exactly what recomputing it would
+          // give up to one more bf16 rounding.
+          float beta = 1.f;
+          if (resc_b) {
+            // A row whose max was still -inf has all-zero P for keys 0-63.
+            beta = m_run == -INFINITY ? 0.f : ex2_approx(m_use - m23 * sl2);
+            m_run = m23 * sl2;
+            m_use = m_run;
+            resc = true;
+          }
+          tmem_st_wait();   // the P just stored is read back
+          rescale_p_half(tS, beta);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          softmax_chunk(s, 2 * h, sl2, m_use, tS, ls);
-          softmax_chunk(s, 2 * h + 1, sl2, m_use, tS, ls);
-          if (h == 0) {
-            if (rescale_o) {
-              // O holds the previous PV products (complete: this tile's s_full was
-              // committed after them) and no PV of this tile starts before
-              // p_full: rescale it in place.
+          for (int q = 0; q < 8; ++q) ls[q] *= beta;
+        }
+        const float alpha = resc ? ex2_approx(m_prev - m_run) : 1.f;   // 0 when m_prev = -inf
+        l_run *= alpha;
+        if (ntile > 0 && __any_sync(0xffffffffu, resc)) {
+          // O holds the previous PV products (complete: this tile's s_full was
+          // committed after them) and no PV of this tile starts before p_full:
+          // rescale it in place.
 #pragma unroll
-              for (int c = 0; c < D; c += 16) {
-                uint32_t o[16];
-                tmem_ld16(tO + c, o);
+          for (int c = 0; c < D; c += 16) {
+            uint32_t o[16];
+            tmem_ld16(tO + c, o);
 #pragma unroll
-                for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-                tmem_st16(tO + c, o);
-              }
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(smem_addr(&sm.p_full[wg][0]));
+            for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+            tmem_st16(tO + c, o);
           }
         }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(smem_addr(&sm.p_full[wg][0]));
+        softmax_chunk(s, 2, sl2, m_use, tS, ls);
+        softmax_chunk(s, 3, sl2, m_use, tS, ls);
         const float lsum = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         l_run += lsum;
         tmem_st_wait();

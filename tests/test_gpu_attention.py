@@ -110,3 +110,25 @@ def test_repeated_calls_are_identical():
     o2, l2 = cp.attn_fwd(plan, qd, kd, vd)
     assert cp.check(plan) == 0
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def _spiked_qkv(B, H, S, D, seed):
+    """Scores with planted maxima that keep growing along the sequence: every
+    query has a constant component along dimension 0 and every 97th key a large,
+    increasing one there, so the running row max jumps by more than 2^8 (in the
+    exp2 domain) many times, in the first and the second half of key tiles."""
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, S, H, D, generator=g)
+    k = torch.randn(B, S, H, D, generator=g)
+    v = torch.randn(B, S, H, D, generator=g)
+    q[..., 0] = 4.0
+    pos = torch.arange(5, S, 97)
+    k[:, pos, :, 0] = (20.0 + 16.0 * torch.arange(len(pos), dtype=torch.float32))[None, :, None]
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("layout,causal,D", [("zigzag", True, 128), ("contiguous", True, 128),
+                                             ("contiguous", False, 128), ("zigzag", True, 64)])
+def test_growing_row_max_rescales(layout, causal, D):
+    q, k, v = _spiked_qkv(1, 2, 2048, D, 21)
+    run_and_compare(q, k, v, 2, layout, causal, what=f"spiked {layout} causal={causal} D={D}")
