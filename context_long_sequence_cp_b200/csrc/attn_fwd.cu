@@ -89,6 +89,11 @@ __device__ __forceinline__ WorkItem ld_item_volatile(const WorkItem* ptr) {
   return WorkItem{v.x, v.y, v.z, v.w};
 }
 
+// One CTA per SM: the dynamic shared memory request (struct + alignment slack)
+// stays within the 227 KB a CTA may use.
+static_assert(sizeof(Smem<128>) + 1024 <= 232448, "Smem<128> exceeds the per-CTA limit");
+static_assert(sizeof(Smem<64>) + 1024 <= 232448, "Smem<64> exceeds the per-CTA limit");
+
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 template <int D>
