@@ -347,11 +347,12 @@ def main():
     prof = os.path.join(ROOT, "profiles", "attn_fwd_zigzag_32k_traffic.json")
     if os.path.exists(prof):
         # DRAM bytes of one launch from an ncu capture, valid only for the kernel
-        # source it was taken on (null once the kernel changed).
+        # and schedule source it was taken on (null once either changed: the
+        # plan's item order decides how much of K/V the L2 serves).
         import hashlib
         csrc = os.path.join(ROOT, "context_long_sequence_cp_b200", "csrc")
         h = hashlib.sha256()
-        for name in ("attn_fwd.cu", "sm100.cuh", "geometry.h"):
+        for name in ("attn_fwd.cu", "sm100.cuh", "geometry.h", "api.cu"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(f.read())
         with open(prof) as f:
