@@ -16,10 +16,11 @@ Contents:
     Ulysses sequence-shard <-> head-group run maps, as int64 index arrays.
   * ``schedule``   — brute-force (query tile, key tile) pair classification and
     per-rank executed tile counts.
+  * ``rope``       — rotary position embedding at global positions.
 
 Every function is pinned by ``tests/test_oracle_*.py`` against something other
 than itself (library special cases, closed forms, invariants, hand-derived
 worked examples under ``tests/golden/``). No function here is "parity
 unpinned".
 """
-from . import attention, layouts, schedule  # noqa: F401
+from . import attention, layouts, rope, schedule  # noqa: F401
