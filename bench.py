@@ -292,6 +292,18 @@ def main():
     perm = statistics.median(perm_ms)
     perm_gbs = 2 * q.numel() * 2 / (perm * 1e-3) / 1e9
 
+    # --- RoPE fused into the same layout map (HBM-bound, same algorithmic bytes)
+    rope_ms = []
+    for _ in range(5):
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        cp.rope_permute(plan, q, out=qz)
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        rope_ms.append(a0.elapsed_time(a1))
+    rope = statistics.median(rope_ms)
+    rope_gbs = 2 * q.numel() * 2 / (rope * 1e-3) / 1e9
+
     # --- unfused path: per-step partials + merge kernel
     op = torch.empty(N, plan.rows, D, dtype=torch.float32, device=dev)
     lp = torch.empty(N, plan.rows, dtype=torch.float32, device=dev)
@@ -375,6 +387,8 @@ def main():
         "components": {
             "attention_ms": att, "attention_tflops": att_tflops,
             "permute_ms": perm, "permute_gbs": perm_gbs, "permute_frac_hbm": perm_gbs / float(peaks["hbm_gbs"]),
+            "rope_permute_ms": rope, "rope_permute_gbs": rope_gbs,
+            "rope_permute_frac_hbm": rope_gbs / float(peaks["hbm_gbs"]),
             "partials_ms": part_ms, "merge_ms": merge_ms, "merge_gbs": merge_gbs,
             "merge_frac_hbm": merge_gbs / float(peaks["hbm_gbs"]),
             "unfused_tflops": w.flops / ((part_ms + merge_ms) * 1e-3) / 1e12,

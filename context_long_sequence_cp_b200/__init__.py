@@ -36,6 +36,7 @@ SIGNATURES = {
     "cp_attn_fwd_partials": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "cp_merge_partials": (_I, [_I, _I64, _I, _P, _P, _P, _P, _P]),
     "cp_layout_permute": (_I, [_P, _I, _P, _P, _I, _P]),
+    "cp_rope_permute": (_I, [_P, _P, _P, ctypes.c_double, _I64, _P]),
     "cp_layout_index_map_len": (_I64, [_P]),
     "cp_layout_index_map": (_I, [_P, _P, _P]),
     "cp_attn_check": (_I, [_P, _P]),
@@ -191,6 +192,22 @@ def layout_permute(plan: Plan, x, direction: int, out=None, stream=None):
         out = torch.empty_like(x)
     _check("cp_layout_permute", lib().cp_layout_permute(plan.handle, int(direction), _ptr(x), _ptr(out),
                                                         x.element_size(), _stream(stream)))
+    return out
+
+
+def rope_permute(plan: Plan, x, out=None, base: float = 10000.0, pos_offset: int = 0, stream=None):
+    """``cp_rope_permute``: rotary embedding at global positions fused into the
+    forward layout map (natural or Ulysses shards -> the attention input layout)."""
+    if x.dtype != torch.bfloat16:
+        raise CpAttnError("cp_rope_permute", -1)
+    if out is None:
+        if plan.layout == "ulysses":
+            B, H, S, D, N = plan.B, plan.H, plan.S, plan.D, plan.N
+            out = torch.empty(N, B, S, H // N, D, dtype=x.dtype, device=x.device)
+        else:
+            out = torch.empty_like(x)
+    _check("cp_rope_permute", lib().cp_rope_permute(plan.handle, _ptr(x), _ptr(out), float(base), int(pos_offset),
+                                                    _stream(stream)))
     return out
 
 

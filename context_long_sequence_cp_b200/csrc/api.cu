@@ -449,6 +449,25 @@ int cp_layout_permute(cp_attn_plan_t plan, int direction, const void* in, void* 
   return launch_permute(a, in, out, static_cast<cudaStream_t>(stream)) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
+int cp_rope_permute(cp_attn_plan_t plan, const void* in, void* out, double base, int64_t pos_offset,
+                    cp_stream_t stream) {
+  if (plan == nullptr || in == nullptr || out == nullptr) return CP_ERR_INVALID_ARG;
+  if (!(base > 1.0) || !std::isfinite(base)) return CP_ERR_INVALID_ARG;
+  if (pos_offset < 0 || pos_offset > (int64_t(1) << 31) - plan->S) return CP_ERR_INVALID_ARG;
+  if (!aligned16(in) || !aligned16(out)) return CP_ERR_ALIGNMENT;
+  if (plan->D % 8 != 0 || plan->D > 128 || 256 % plan->D != 0) return CP_ERR_UNSUPPORTED;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) return CP_ERR_CUDA;
+  RopeArgs ra;
+  std::memset(&ra, 0, sizeof(ra));
+  for (int i = 0; i < plan->D / 2; ++i) ra.theta[i] = std::pow(base, -2.0 * i / plan->D);
+  ra.pos_offset = pos_offset;
+  ra.D = plan->D;
+  return launch_rope_permute(permute_args(plan, 0, 2), ra, in, out, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? CP_OK
+             : CP_ERR_CUDA;
+}
+
 int64_t cp_layout_index_map_len(cp_attn_plan_t plan) {
   if (plan == nullptr) return CP_ERR_INVALID_ARG;
   return plan->layout == CP_LAYOUT_ULYSSES ? static_cast<int64_t>(plan->N) * plan->B * plan->S

@@ -58,6 +58,15 @@ struct PermuteArgs {
 cudaError_t launch_permute(const PermuteArgs& a, const void* in, void* out, cudaStream_t stream);
 cudaError_t launch_index_map(const PermuteArgs& a, int64_t* map_out, cudaStream_t stream);
 
+// Rotary embedding parameters: theta[i] = base^(-2i/D) (fp64), i < D/2 <= 64.
+struct RopeArgs {
+  double theta[64];
+  int64_t pos_offset;
+  int D;
+};
+cudaError_t launch_rope_permute(const PermuteArgs& a, const RopeArgs& ra, const void* in, void* out,
+                                cudaStream_t stream);
+
 // probe.cu
 cudaError_t launch_wait_probe(int* status, uint64_t limit_ns, cudaStream_t stream);
 

@@ -154,6 +154,54 @@ __global__ void __launch_bounds__(256) permute_kernel(UnitMap m, int64_t units, 
   }
 }
 
+// Rotary position embedding fused into the forward gather (natural or Ulysses
+// shards -> the attention view). Page "序列与上下文并行" (ai-infra-wiki), section
+// "工程实践": under CP the position encoding of a token is computed at its GLOBAL
+// position. Feature pair (2i, 2i+1) of every head at global position p is
+// rotated by p * theta_i, theta_i = base^(-2i/D) (the frequencies of the pages'
+// sinusoidal PositionalEncoding). The global position of an output unit is its
+// natural token index (source row mod S for token rows; output run mod S for
+// Ulysses head-group runs) plus pos_offset.
+//
+// The angle and its reduction to [-pi, pi] are computed in fp64 (positions up to
+// 2^31 keep full fp32 accuracy of the reduced angle), then sincosf. A warp's 32
+// lanes x 8 bf16 span whole heads (D in {64, 128}), so every lane always holds
+// the same four feature pairs: it takes their cos/sin once per unit and applies
+// them to all its 16-byte vectors.
+__global__ void __launch_bounds__(256) rope_permute_kernel(UnitMap m, int64_t units, int vec_per_unit, RopeArgs ra,
+                                                           const uint4* __restrict__ in, uint4* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int i0 = ((8 * lane) % ra.D) / 2;   // first feature pair of this lane's vectors
+  constexpr double kTwoPi = 6.283185307179586476925286766559;
+  constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+  for (int64_t u = warp0; u < units; u += nwarps) {
+    const int64_t s = m.src(u);
+    const int64_t p = (m.kind == 0 ? s % m.S : u % m.S) + ra.pos_offset;
+    float c[4], sn[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const double a = static_cast<double>(p) * ra.theta[i0 + k];
+      const double r = a - rint(a * kInvTwoPi) * kTwoPi;
+      sincosf(static_cast<float>(r), &sn[k], &c[k]);
+    }
+    const uint4* src = in + s * vec_per_unit;
+    uint4* dst = out + u * vec_per_unit;
+    for (int v = lane; v < vec_per_unit; v += 32) {
+      const uint4 x = __ldg(src + v);
+      uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float xe = __uint_as_float(w[k] << 16);          // feature 2i
+        const float xo = __uint_as_float(w[k] & 0xffff0000u);  // feature 2i+1
+        w[k] = sm100::pack_bf16x2(xe * c[k] - xo * sn[k], xe * sn[k] + xo * c[k]);
+      }
+      dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
 __global__ void index_map_kernel(UnitMap m, int64_t units, int64_t* __restrict__ map) {
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < units; i += stride)
@@ -213,6 +261,20 @@ cudaError_t launch_permute(const PermuteArgs& a, const void* in, void* out, cuda
   if (blocks > cap) blocks = cap;
   permute_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(make_map(a), units, vpu,
                                                                static_cast<const uint4*>(in), static_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_permute(const PermuteArgs& a, const RopeArgs& ra, const void* in, void* out,
+                                cudaStream_t stream) {
+  const int64_t units = a.kind == 0 ? static_cast<int64_t>(a.B) * a.S : static_cast<int64_t>(a.N) * a.B * a.S;
+  if (units == 0) return cudaSuccess;
+  const int64_t unit_elems = (static_cast<int64_t>(a.B) * a.S * a.H * a.D) / units;
+  const int vpu = static_cast<int>(unit_elems / 8);   // 16-byte vectors of bf16
+  int64_t blocks = (units + 7) / 8;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  if (blocks > cap) blocks = cap;
+  rope_permute_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(
+      make_map(a), units, vpu, ra, static_cast<const uint4*>(in), static_cast<uint4*>(out));
   return cudaGetLastError();
 }
 

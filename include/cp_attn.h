@@ -192,6 +192,33 @@ CP_API int cp_merge_partials(int num_parts, int64_t rows, int D, const float* o_
 CP_API int cp_layout_permute(cp_attn_plan_t plan, int direction, const void* in, void* out,
                       int elem_bytes, cp_stream_t stream);
 
+/*
+ * Rotary position embedding at GLOBAL positions, fused into the forward layout
+ * map. Page "序列与上下文并行" (ai-infra-wiki), section "工程实践": under context
+ * parallelism position encodings are computed at each token's global position
+ * (each rank must know its segment's global offset). Reading: feature pair
+ * (2i, 2i+1) of every head of the token at global position p is rotated by the
+ * angle p * theta_i, theta_i = base^(-2i/D) — the frequencies of the pages'
+ * sinusoidal PositionalEncoding (page "Tensor并行与算子拆分"); base 10000 there:
+ *   out[2i]   = in[2i] cos - in[2i+1] sin,   out[2i+1] = in[2i] sin + in[2i+1] cos.
+ *
+ * in:  bf16 device memory in the natural layout [B][S][H][D] (contiguous and
+ *      zigzag plans) or the Ulysses sequence shards [N][B][S/N][H][D]; the global
+ *      position of a token is its natural index s (shard rho, local sl: rho*S/N + sl)
+ *      plus pos_offset (the position of token 0, e.g. after a cached prefix).
+ * out: bf16 device memory in the plan's attention input layout, exactly what
+ *      cp_layout_permute(plan, 0, in, out, 2) writes, with every head rotated:
+ *      zigzag/contiguous rank-major [N][B][S/N][H][D]; for Ulysses the head
+ *      groups [N][B][S][H/N][D] that cp_attn_fwd builds internally.
+ * base > 1 (10000 for the pages' frequencies); 0 <= pos_offset <= 2^31 - S.
+ * The angle is reduced to [-pi, pi] in fp64, then rotated in fp32; one bf16
+ * rounding per output element. Enqueued on `stream`; `in` and `out` must not
+ * overlap; both 16-byte aligned (CP_ERR_ALIGNMENT); bad arguments give
+ * CP_ERR_INVALID_ARG; D must be 64 or 128 (CP_ERR_UNSUPPORTED).
+ */
+CP_API int cp_rope_permute(cp_attn_plan_t plan, const void* in, void* out, double base, int64_t pos_offset,
+                           cp_stream_t stream);
+
 /* Length of the index map written by cp_layout_index_map: B*S for
  * contiguous/zigzag (one entry per token), N*B*S for Ulysses (one entry per
  * (group, batch, token) run of H/N heads). */

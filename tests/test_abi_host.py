@@ -156,3 +156,21 @@ def test_static_schedule_small_plan_one_item_per_cta():
     assert len(loads) == p.num_items() == 8
     # Non-causal: every item walks all 4 ranks' single key tile.
     assert loads == [2 * 4 + 3] * 8
+
+
+def test_rope_permute_argument_validation():
+    # Host-side checks run before any device work (no GPU here: valid calls end
+    # in CP_ERR_CUDA).
+    L = cp.lib()
+    p = cp.Plan(1, 2, 256, 64, 4, True, "zigzag")
+    ok_in, ok_out = ctypes.c_void_p(4096), ctypes.c_void_p(8192)
+    assert L.cp_rope_permute(None, ok_in, ok_out, 10000.0, 0, None) == -1
+    assert L.cp_rope_permute(p.handle, None, ok_out, 10000.0, 0, None) == -1
+    assert L.cp_rope_permute(p.handle, ok_in, None, 10000.0, 0, None) == -1
+    assert L.cp_rope_permute(p.handle, ok_in, ok_out, 1.0, 0, None) == -1        # base must be > 1
+    assert L.cp_rope_permute(p.handle, ok_in, ok_out, float("nan"), 0, None) == -1
+    assert L.cp_rope_permute(p.handle, ok_in, ok_out, 10000.0, -1, None) == -1   # negative offset
+    assert L.cp_rope_permute(p.handle, ok_in, ok_out, 10000.0, (1 << 31) - 255, None) == -1
+    assert L.cp_rope_permute(p.handle, ctypes.c_void_p(4100), ok_out, 10000.0, 0, None) == -3   # alignment
+    assert L.cp_rope_permute(p.handle, ok_in, ok_out, 10000.0, (1 << 31) - 256, None) in (0, -4)
+    p.close()
