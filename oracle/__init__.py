@@ -17,10 +17,12 @@ Contents:
   * ``schedule``   — brute-force (query tile, key tile) pair classification and
     per-rank executed tile counts.
   * ``rope``       — rotary position embedding at global positions.
+  * ``attention_bwd`` — gradients of softmax attention (dQ, dK, dV), by the
+    chain rule on the forward's definition.
 
 Every function is pinned by ``tests/test_oracle_*.py`` against something other
 than itself (library special cases, closed forms, invariants, hand-derived
 worked examples under ``tests/golden/``). No function here is "parity
 unpinned".
 """
-from . import attention, layouts, rope, schedule  # noqa: F401
+from . import attention, attention_bwd, layouts, rope, schedule  # noqa: F401
