@@ -31,6 +31,9 @@ SIGNATURES = {
     "cp_attn_plan_tile_counts": (_I64, [_P, _P]),
     "cp_attn_plan_num_items": (_I64, [_P]),
     "cp_attn_plan_cta_loads": (_I64, [_P, _P]),
+    "cp_attn_bwd": (_I, [_P] * 12),
+    "cp_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_P]),
+    "cp_attn_plan_bwd_pairs": (_I64, [_P, _P, _P]),
     "cp_attn_workspace_bytes": (_SZ, [_P, _I]),
     "cp_attn_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "cp_attn_fwd_partials": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
@@ -128,6 +131,17 @@ class Plan:
     def num_items(self) -> int:
         return int(lib().cp_attn_plan_num_items(self._h))
 
+    def bwd_pairs(self):
+        """(key-tile walk pairs, query-tile walk pairs) of the backward, per (batch, head)."""
+        kv, qq = ctypes.c_int64(0), ctypes.c_int64(0)
+        rc = int(lib().cp_attn_plan_bwd_pairs(self._h, ctypes.byref(kv), ctypes.byref(qq)))
+        if rc < 0:
+            raise CpAttnError("cp_attn_plan_bwd_pairs", rc)
+        return int(kv.value), int(qq.value)
+
+    def bwd_workspace_bytes(self) -> int:
+        return int(lib().cp_attn_bwd_workspace_bytes(self._h))
+
     def cta_loads(self):
         """Modelled load of each CTA of the kernel's static schedule."""
         n = int(lib().cp_attn_plan_cta_loads(self._h, None))
@@ -209,6 +223,18 @@ def rope_permute(plan: Plan, x, out=None, base: float = 10000.0, pos_offset: int
     _check("cp_rope_permute", lib().cp_rope_permute(plan.handle, _ptr(x), _ptr(out), float(base), int(pos_offset),
                                                     _stream(stream)))
     return out
+
+
+def attn_bwd(plan: Plan, q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """``cp_attn_bwd``: (dq, dk, dv) in the plan's attention input layout."""
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(max(plan.bwd_workspace_bytes(), 16), dtype=torch.uint8, device=q.device)
+    _check("cp_attn_bwd", lib().cp_attn_bwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                            _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), _stream(stream)))
+    return dq, dk, dv
 
 
 def layout_index_map(plan: Plan, device="cuda", stream=None):

@@ -13,6 +13,7 @@
 #include <utility>
 #include <vector>
 
+#include "attn_bwd.h"
 #include "attn_fwd.h"
 #include "cp_attn.h"
 #include "geometry.h"
@@ -42,6 +43,23 @@ struct cp_attn_plan_s {
   std::vector<int> cta_begin;
   std::vector<int64_t> cta_load;    // modelled cost per CTA (key tiles + item overhead)
   int* d_cta_begin = nullptr;
+  // Backward schedules (contiguous and zigzag layouts): per key tile the query
+  // tiles that see it (dK/dV kernel), per query tile the key tiles it sees (dQ
+  // kernel); walks are per (rank, tile), shared by every batch and head.
+  struct BwdSched {
+    std::vector<WorkItem> items;
+    std::vector<int> cta_begin;
+    std::vector<int64_t> cta_load;
+    std::vector<int> walk_off;        // NR * ntiles + 1
+    std::vector<uint32_t> entries;    // pack_entry(other rank, other tile, class, 0)
+    int n_cta = 0;
+    WorkItem* d_items = nullptr;
+    int* d_cta_begin = nullptr;
+    int* d_walk_off = nullptr;
+    uint32_t* d_entries = nullptr;
+  };
+  int ntiles = 0;
+  BwdSched bwd_kv, bwd_q;
 };
 
 namespace {
@@ -107,6 +125,40 @@ constexpr int64_t kItemOverheadHalfTiles = 3;
 // lower index). Items therefore start in about list order (so that the items
 // running together still share keys and values in L2) while the CTAs finish
 // together. The list is reordered so that each CTA's items are contiguous.
+// Assigns a sorted work list to n_cta persistent CTAs: each item, in list order,
+// goes to the CTA whose modelled finish time is the earliest (ties to the lower
+// index). Items therefore start in about list order (so that the items running
+// together still share their operands in L2) while the CTAs finish together.
+// The list is reordered so that each CTA's items are contiguous.
+int assign_greedy(std::vector<WorkItem>& items, const std::vector<int64_t>& cost, int n_cta,
+                  std::vector<int>& cta_begin, std::vector<int64_t>& cta_load) {
+  const int n = static_cast<int>(items.size());
+  n_cta = n < n_cta ? n : n_cta;
+  cta_load.assign(n_cta, 0);
+  std::vector<int> owner(n);
+  using Slot = std::pair<int64_t, int>;
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> free_at;
+  for (int c = 0; c < n_cta; ++c) free_at.push(Slot(0, c));
+  for (int i = 0; i < n; ++i) {
+    const Slot s = free_at.top();
+    free_at.pop();
+    owner[i] = s.second;
+    cta_load[s.second] = s.first + cost[i];
+    free_at.push(Slot(s.first + cost[i], s.second));
+  }
+  std::vector<WorkItem> sorted;
+  sorted.reserve(n);
+  cta_begin.assign(n_cta + 1, 0);
+  for (int c = 0; c < n_cta; ++c) {
+    cta_begin[c] = static_cast<int>(sorted.size());
+    for (int i = 0; i < n; ++i)
+      if (owner[i] == c) sorted.push_back(items[i]);
+  }
+  cta_begin[n_cta] = n;
+  items.swap(sorted);
+  return n_cta;
+}
+
 void schedule_items(cp_attn_plan_s* p, int n_cta) {
   const int n = static_cast<int>(p->items.size());
   std::vector<int64_t> cost(n);
@@ -116,30 +168,79 @@ void schedule_items(cp_attn_plan_s* p, int n_cta) {
     const int* off = p->step_off.data() + static_cast<size_t>(rq * p->npairs + w.qp) * (p->g.NR + 1);
     cost[i] = 2 * static_cast<int64_t>(off[p->g.NR] - off[0]) + kItemOverheadHalfTiles;
   }
-  n_cta = n < n_cta ? n : n_cta;
-  p->n_cta = n_cta;
-  p->cta_load.assign(n_cta, 0);
-  std::vector<int> owner(n);
-  using Slot = std::pair<int64_t, int>;
-  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> free_at;
-  for (int c = 0; c < n_cta; ++c) free_at.push(Slot(0, c));
-  for (int i = 0; i < n; ++i) {
-    const Slot s = free_at.top();
-    free_at.pop();
-    owner[i] = s.second;
-    p->cta_load[s.second] = s.first + cost[i];
-    free_at.push(Slot(s.first + cost[i], s.second));
+  p->n_cta = assign_greedy(p->items, cost, n_cta, p->cta_begin, p->cta_load);
+}
+
+// Walks and schedules of the two backward kernels. A walk entry's class is
+// kFull when every (row, column) pair of the tile pair is allowed and both tiles
+// are whole; otherwise kMasked (the kernels then bound the allowed columns).
+void build_bwd(cp_attn_plan_s* p, int n_cta) {
+  const Geometry& g = p->g;
+  const int nt = (g.T + kTile - 1) / kTile;
+  p->ntiles = nt;
+  for (int kind = 0; kind < 2; ++kind) {   // 0: dK/dV (per key tile), 1: dQ (per query tile)
+    cp_attn_plan_s::BwdSched& b = kind == 0 ? p->bwd_kv : p->bwd_q;
+    b.walk_off.assign(static_cast<size_t>(g.NR) * nt + 1, 0);
+    b.entries.clear();
+    for (int r = 0; r < g.NR; ++r) {
+      for (int tile = 0; tile < nt; ++tile) {
+        b.walk_off[static_cast<size_t>(r) * nt + tile] = static_cast<int>(b.entries.size());
+        for (int t = 0; t < g.NR; ++t) {
+          // dK/dV: the query ranks whose ring step t reaches key rank r; dQ: the
+          // key rank of step t of query rank r.
+          const int other = kind == 0 ? (r - t + g.NR) % g.NR : (r + t) % g.NR;
+          for (int ot = 0; ot < nt; ++ot) {
+            const int rq = kind == 0 ? other : r, qt = kind == 0 ? ot : tile;
+            const int rk = kind == 0 ? r : other, kt = kind == 0 ? tile : ot;
+            int c = classify(g, rq, qt * kTile, rk, kt * kTile);
+            if (c == kSkip) continue;
+            if (c == kFull && g.T - qt * kTile < kTile) c = kMasked;   // ragged query tile
+            b.entries.push_back(pack_entry(other, ot, c, 0));
+          }
+        }
+      }
+    }
+    b.walk_off[static_cast<size_t>(g.NR) * nt] = static_cast<int>(b.entries.size());
+    b.items.clear();
+    for (int r = 0; r < g.NR; ++r)
+      for (int bb = 0; bb < g.B; ++bb)
+        for (int tile = 0; tile < nt; ++tile) {
+          const int len = b.walk_off[static_cast<size_t>(r) * nt + tile + 1] - b.walk_off[static_cast<size_t>(r) * nt + tile];
+          for (int h = 0; h < g.Hh; ++h) b.items.push_back(WorkItem{r * g.B + bb, h, tile, len});
+        }
+    std::stable_sort(b.items.begin(), b.items.end(), [&](const WorkItem& x, const WorkItem& y) {
+      const int bx = x.rb % g.B, by = y.rb % g.B;
+      if (bx != by) return bx < by;
+      if (x.h / 2 != y.h / 2) return x.h / 2 < y.h / 2;
+      return x.cost > y.cost;
+    });
+    std::vector<int64_t> cost(b.items.size());
+    for (size_t i = 0; i < b.items.size(); ++i) cost[i] = 2 * static_cast<int64_t>(b.items[i].cost) + kItemOverheadHalfTiles;
+    b.n_cta = assign_greedy(b.items, cost, n_cta, b.cta_begin, b.cta_load);
   }
-  std::vector<WorkItem> sorted;
-  sorted.reserve(n);
-  p->cta_begin.assign(n_cta + 1, 0);
-  for (int c = 0; c < n_cta; ++c) {
-    p->cta_begin[c] = static_cast<int>(sorted.size());
-    for (int i = 0; i < n; ++i)
-      if (owner[i] == c) sorted.push_back(p->items[i]);
-  }
-  p->cta_begin[n_cta] = n;
-  p->items.swap(sorted);
+}
+
+bool upload_bwd(cp_attn_plan_s::BwdSched& b) {
+  const size_t ib = b.items.size() * sizeof(WorkItem), cb = b.cta_begin.size() * sizeof(int);
+  const size_t wb = b.walk_off.size() * sizeof(int), eb = b.entries.size() * sizeof(uint32_t);
+  return cudaMalloc(&b.d_items, ib > 0 ? ib : sizeof(WorkItem)) == cudaSuccess &&
+         cudaMalloc(&b.d_cta_begin, cb) == cudaSuccess && cudaMalloc(&b.d_walk_off, wb) == cudaSuccess &&
+         cudaMalloc(&b.d_entries, eb > 0 ? eb : sizeof(uint32_t)) == cudaSuccess &&
+         (ib == 0 || cudaMemcpy(b.d_items, b.items.data(), ib, cudaMemcpyHostToDevice) == cudaSuccess) &&
+         cudaMemcpy(b.d_cta_begin, b.cta_begin.data(), cb, cudaMemcpyHostToDevice) == cudaSuccess &&
+         cudaMemcpy(b.d_walk_off, b.walk_off.data(), wb, cudaMemcpyHostToDevice) == cudaSuccess &&
+         (eb == 0 || cudaMemcpy(b.d_entries, b.entries.data(), eb, cudaMemcpyHostToDevice) == cudaSuccess);
+}
+
+void free_bwd(cp_attn_plan_s::BwdSched& b) {
+  if (b.d_items != nullptr) cudaFree(b.d_items);
+  if (b.d_cta_begin != nullptr) cudaFree(b.d_cta_begin);
+  if (b.d_walk_off != nullptr) cudaFree(b.d_walk_off);
+  if (b.d_entries != nullptr) cudaFree(b.d_entries);
+  b.d_items = nullptr;
+  b.d_cta_begin = nullptr;
+  b.d_walk_off = nullptr;
+  b.d_entries = nullptr;
 }
 
 int ensure_device(cp_attn_plan_s* p) {
@@ -296,6 +397,7 @@ int cp_attn_plan(cp_attn_plan_t* out, int B, int H, int S, int D, int N, int cau
       sms = kDefaultSmCount;
   }
   schedule_items(p, sms);
+  if (layout != CP_LAYOUT_ULYSSES) build_bwd(p, sms);
   if (have_device) {
     const size_t bytes = p->items.size() * sizeof(WorkItem);
     const size_t off_bytes = p->step_off.size() * sizeof(int);
@@ -311,8 +413,11 @@ int cp_attn_plan(cp_attn_plan_t* out, int B, int H, int S, int D, int N, int cau
               cudaMemcpy(p->d_step_off, p->step_off.data(), off_bytes, cudaMemcpyHostToDevice) == cudaSuccess &&
               (ent_bytes == 0 ||
                cudaMemcpy(p->d_entries, p->entries.data(), ent_bytes, cudaMemcpyHostToDevice) == cudaSuccess) &&
-              cudaMemset(p->d_status, 0, sizeof(int)) == cudaSuccess;
+              cudaMemset(p->d_status, 0, sizeof(int)) == cudaSuccess &&
+              (layout == CP_LAYOUT_ULYSSES || (upload_bwd(p->bwd_kv) && upload_bwd(p->bwd_q)));
     if (!ok) {
+      free_bwd(p->bwd_kv);
+      free_bwd(p->bwd_q);
       cudaFree(p->d_items);
       cudaFree(p->d_cta_begin);
       p->d_cta_begin = nullptr;
@@ -335,6 +440,8 @@ int cp_attn_plan_destroy(cp_attn_plan_t plan) {
   if (plan == nullptr) return CP_OK;
   if (plan->d_items != nullptr) cudaFree(plan->d_items);
   if (plan->d_cta_begin != nullptr) cudaFree(plan->d_cta_begin);
+  free_bwd(plan->bwd_kv);
+  free_bwd(plan->bwd_q);
   if (plan->d_status != nullptr) cudaFree(plan->d_status);
   if (plan->d_step_off != nullptr) cudaFree(plan->d_step_off);
   if (plan->d_entries != nullptr) cudaFree(plan->d_entries);
@@ -355,6 +462,84 @@ int64_t cp_attn_plan_tile_counts(cp_attn_plan_t plan, int64_t* per_rank) {
 int64_t cp_attn_plan_num_items(cp_attn_plan_t plan) {
   if (plan == nullptr) return CP_ERR_INVALID_ARG;
   return static_cast<int64_t>(plan->items.size());
+}
+
+size_t cp_attn_bwd_workspace_bytes(cp_attn_plan_t plan) {
+  if (plan == nullptr || plan->layout == CP_LAYOUT_ULYSSES) return 0;
+  const int64_t rows = static_cast<int64_t>(plan->g.NR) * plan->g.B * plan->g.T * plan->g.Hh;
+  return static_cast<size_t>(2 * rows * 4 + 1024);   // lse2 and dvec, plus bulk-copy over-read padding
+}
+
+int64_t cp_attn_plan_bwd_pairs(cp_attn_plan_t plan, int64_t* kv_pairs, int64_t* q_pairs) {
+  if (plan == nullptr) return CP_ERR_INVALID_ARG;
+  if (plan->layout == CP_LAYOUT_ULYSSES) return CP_ERR_UNSUPPORTED;
+  if (kv_pairs != nullptr) *kv_pairs = static_cast<int64_t>(plan->bwd_kv.entries.size());
+  if (q_pairs != nullptr) *q_pairs = static_cast<int64_t>(plan->bwd_q.entries.size());
+  return static_cast<int64_t>(plan->bwd_q.entries.size());
+}
+
+int cp_attn_bwd(cp_attn_plan_t plan, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                const void* dout, void* dq, void* dk, void* dv, void* workspace, cp_stream_t stream) {
+  if (plan == nullptr || q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr ||
+      dout == nullptr || dq == nullptr || dk == nullptr || dv == nullptr || workspace == nullptr)
+    return CP_ERR_INVALID_ARG;
+  if (plan->layout == CP_LAYOUT_ULYSSES) return CP_ERR_UNSUPPORTED;
+  if (plan->g.T % 4 != 0) return CP_ERR_UNSUPPORTED;   // 16-byte rows of the per-row statistics
+  const void* ptrs[11] = {q, k, v, o, lse, dout, dq, dk, dv, workspace, nullptr};
+  for (int i = 0; i < 10; ++i)
+    if (!aligned16(ptrs[i])) return CP_ERR_ALIGNMENT;
+  if (plan->d_items == nullptr || plan->bwd_kv.d_items == nullptr) return CP_ERR_CUDA;
+  const Geometry& g = plan->g;
+  const int64_t rows = static_cast<int64_t>(g.NR) * g.B * g.T * g.Hh;
+  float* lse2 = static_cast<float*>(workspace);
+  float* dvec = lse2 + rows;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  BwdPreParams pre;
+  pre.g = g;
+  pre.o = static_cast<const __nv_bfloat16*>(o);
+  pre.dout = static_cast<const __nv_bfloat16*>(dout);
+  pre.lse = lse;
+  pre.lse_B = plan->lse_B;
+  pre.lse_H = plan->lse_H;
+  pre.lse_S = plan->lse_S;
+  pre.lse2 = lse2;
+  pre.dvec = dvec;
+  if (launch_attn_bwd_pre(pre, plan->D, st) != cudaSuccess) return CP_ERR_CUDA;
+
+  BwdLaunch L;
+  std::memset(&L, 0, sizeof(L));
+  int rc;
+  if ((rc = encode_view(&L.tm_q, q, g, plan->D)) != CP_OK) return rc;
+  if ((rc = encode_view(&L.tm_k, k, g, plan->D)) != CP_OK) return rc;
+  if ((rc = encode_view(&L.tm_v, v, g, plan->D)) != CP_OK) return rc;
+  if ((rc = encode_view(&L.tm_do, dout, g, plan->D)) != CP_OK) return rc;
+  BwdParams& P = L.params;
+  P.g = g;
+  P.scale = plan->scale;
+  P.scale_log2 = plan->scale * 1.4426950408889634f;
+  P.ntiles = plan->ntiles;
+  P.lse2 = lse2;
+  P.dvec = dvec;
+  P.status = plan->d_status;
+  P.wait_limit_ns = kWaitLimitNs;
+  P.items = plan->bwd_kv.d_items;
+  P.cta_begin = plan->bwd_kv.d_cta_begin;
+  P.n_cta = plan->bwd_kv.n_cta;
+  P.walk_off = plan->bwd_kv.d_walk_off;
+  P.entries = plan->bwd_kv.d_entries;
+  P.out0 = static_cast<__nv_bfloat16*>(dk);
+  P.out1 = static_cast<__nv_bfloat16*>(dv);
+  if (launch_attn_bwd_kv(L, plan->D, st) != cudaSuccess) return CP_ERR_CUDA;
+  P.items = plan->bwd_q.d_items;
+  P.cta_begin = plan->bwd_q.d_cta_begin;
+  P.n_cta = plan->bwd_q.n_cta;
+  P.walk_off = plan->bwd_q.d_walk_off;
+  P.entries = plan->bwd_q.d_entries;
+  P.out0 = static_cast<__nv_bfloat16*>(dq);
+  P.out1 = nullptr;
+  if (launch_attn_bwd_q(L, plan->D, st) != cudaSuccess) return CP_ERR_CUDA;
+  return CP_OK;
 }
 
 int64_t cp_attn_plan_cta_loads(cp_attn_plan_t plan, int64_t* per_cta) {

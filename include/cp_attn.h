@@ -165,6 +165,43 @@ CP_API int cp_attn_fwd_partials(cp_attn_plan_t plan, const void* q, const void* 
                          cp_stream_t stream);
 
 /*
+ * Backward pass: dQ, dK, dV from the forward's saved O and lse. The pages train
+ * long-context models but print no backward; it is the chain rule of the
+ * forward's softmax attention (page "Tensor并行与算子拆分", section
+ * "注意力的并行化优化"), per (batch, head), with the same global-position causal
+ * mask and ring walk as the forward:
+ *   P = exp(scale Q K^T - lse), dV = P^T dO, dP = dO V^T, Dr = rowsum(dO * O),
+ *   dS = P * (dP - Dr), dQ = scale dS K, dK = scale dS^T Q.
+ *
+ * q, k, v, o, dout, dq, dk, dv: bf16 device memory in the plan's attention input
+ * layout (zigzag or contiguous rank-major [N][B][S/N][H][D]; o as cp_attn_fwd
+ * wrote it); lse: fp32 [B][H][S] natural, as cp_attn_fwd wrote it. workspace:
+ * device memory of cp_attn_bwd_workspace_bytes(plan) bytes (per-row lse and
+ * rowsum(dO * O), caller-owned, overwritten). Three kernels are enqueued on
+ * `stream` (row statistics, dK/dV per key tile, dQ per query tile); nothing is
+ * allocated and nothing synchronises; results are deterministic (no atomics).
+ * Errors: CP_ERR_INVALID_ARG (null argument), CP_ERR_UNSUPPORTED (Ulysses
+ * layout, or S/N not a multiple of 4), CP_ERR_ALIGNMENT (a pointer not 16-byte
+ * aligned), CP_ERR_CUDA (no device / launch failure); a bounded in-kernel wait
+ * that runs out is reported by cp_attn_check as CP_ERR_TIMEOUT.
+ */
+CP_API int cp_attn_bwd(cp_attn_plan_t plan, const void* q, const void* k, const void* v, const void* o,
+                       const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                       cp_stream_t stream);
+
+/* Workspace bytes of cp_attn_bwd (0 for a Ulysses plan, which has no backward). */
+CP_API size_t cp_attn_bwd_workspace_bytes(cp_attn_plan_t plan);
+
+/*
+ * Walk lengths of the backward schedule, per (batch, head): *kv_pairs = the
+ * (key tile, query tile) pairs the dK/dV kernel visits, *q_pairs = the (query
+ * tile, key tile) pairs the dQ kernel visits (either may be NULL). Both equal
+ * the executed tile pairs of the forward. Returns *q_pairs, or a negative status
+ * (CP_ERR_UNSUPPORTED for Ulysses).
+ */
+CP_API int64_t cp_attn_plan_bwd_pairs(cp_attn_plan_t plan, int64_t* kv_pairs, int64_t* q_pairs);
+
+/*
  * Merge num_parts partials per row (same section: online-softmax merge):
  *   M = max_t lse_t, lse = M + ln sum_t exp(lse_t - M), O = sum_t exp(lse_t - lse) O_t.
  * Partials with lse_t = -inf contribute nothing; rows whose partials are all

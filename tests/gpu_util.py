@@ -29,6 +29,16 @@ def to_layout(x: torch.Tensor, N: int, layout: str) -> torch.Tensor:
     return x.reshape(B * S, H, D)[m].reshape(N, B, S // N, H, D).contiguous()
 
 
+def from_layout(y: torch.Tensor, N: int, layout: str) -> torch.Tensor:
+    """The layout's tensor [N, B, S/N, H, D] -> natural [B, S, H, D] (inverse of to_layout)."""
+    N_, B, T, H, D = y.shape
+    S = N * T
+    m = torch.from_numpy(token_map(B, S, N, layout)).to(y.device)
+    nat = torch.empty(B * S, H, D, dtype=y.dtype, device=y.device)
+    nat[m] = y.reshape(B * S, H, D)
+    return nat.reshape(B, S, H, D)
+
+
 def gather_rows(o_layout: torch.Tensor, B, S, H, N, layout, rows: np.ndarray) -> np.ndarray:
     """Rows (b, h, i) of a layout-shaped output, as fp64 numpy [n, D]."""
     D = o_layout.shape[-1]

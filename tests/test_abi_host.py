@@ -174,3 +174,39 @@ def test_rope_permute_argument_validation():
     assert L.cp_rope_permute(p.handle, ctypes.c_void_p(4100), ok_out, 10000.0, 0, None) == -3   # alignment
     assert L.cp_rope_permute(p.handle, ok_in, ok_out, 10000.0, (1 << 31) - 256, None) in (0, -4)
     p.close()
+
+
+@pytest.mark.parametrize("S,N,layout,causal", [
+    (32768, 8, "zigzag", True), (4096, 4, "zigzag", True), (800, 4, "contiguous", True),
+    (256, 4, "contiguous", False), (384, 3, "zigzag", True),
+])
+def test_bwd_walks_cover_every_executed_tile_pair(S, N, layout, causal):
+    # Both backward walks visit exactly the executed (query tile, key tile)
+    # pairs of the forward, counted by brute force in the oracle.
+    p = cp.Plan(1, 2, S, 128, N, causal, layout)
+    kv, qq = p.bwd_pairs()
+    ref = int(Sch.tile_pair_counts(S, N, layout, causal).sum())
+    assert kv == qq == ref
+    rows = N * 1 * (S // N) * 2
+    assert p.bwd_workspace_bytes() == 2 * rows * 4 + 1024
+    p.close()
+
+
+def test_bwd_argument_validation():
+    L = cp.lib()
+    p = cp.Plan(1, 2, 256, 64, 4, True, "zigzag")
+    a = [ctypes.c_void_p(4096 * (i + 1)) for i in range(10)]
+    assert L.cp_attn_bwd(None, *a, None) == -1
+    for i in range(10):
+        b = list(a)
+        b[i] = None
+        assert L.cp_attn_bwd(p.handle, *b, None) == -1, i
+    b = list(a)
+    b[3] = ctypes.c_void_p(4100)
+    assert L.cp_attn_bwd(p.handle, *b, None) == -3                  # alignment
+    assert L.cp_attn_bwd(p.handle, *a, None) in (0, -4)             # no device here
+    u = cp.Plan(2, 8, 256, 64, 4, False, "ulysses")
+    assert L.cp_attn_bwd(u.handle, *a, None) == -2                  # no Ulysses backward
+    assert u.bwd_workspace_bytes() == 0
+    p.close()
+    u.close()

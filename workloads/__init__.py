@@ -97,6 +97,14 @@ def make_small(B, H, S, D, seed, scale=1.0, device="cpu"):
     return tuple(out)
 
 
+def make_dout(shape, seed):
+    """Seeded upstream gradient dO for the backward: randn fp32 -> bf16, drawn
+    from its own generator (seed 1000 + seed) in natural [B, S, H, D] order."""
+    g = torch.Generator("cpu")
+    g.manual_seed(1000 + seed)
+    return torch.randn(*shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
 def sample_rows(w: Workload, n: Optional[int] = None) -> np.ndarray:
     """Sampled query rows (b, h, i) in natural coordinates, int64 [n_rows, 3].
 
