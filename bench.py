@@ -304,6 +304,29 @@ def main():
     rope = statistics.median(rope_ms)
     rope_gbs = 2 * q.numel() * 2 / (rope * 1e-3) / 1e9
 
+    # --- backward pass (dQ, dK, dV) on the same inputs; dO seeded like the inputs
+    from workloads import make_dout
+    dod = torch.empty_like(qz)
+    cp.layout_permute(plan, make_dout(q_h.shape, w.seed).to(dev), 0, out=dod)
+    cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=lse)
+    gq, gk, gv = (torch.empty_like(qz) for _ in range(3))
+    bws = torch.empty(plan.bwd_workspace_bytes(), dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        cp.attn_bwd(plan, qz, kz, vz, oz, lse, dod, gq, gk, gv, bws)
+    bwd_ms = []
+    for _ in range(5):
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        cp.attn_bwd(plan, qz, kz, vz, oz, lse, dod, gq, gk, gv, bws)
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        bwd_ms.append(a0.elapsed_time(a1))
+    bwd = statistics.median(bwd_ms)
+    st = cp.check(plan)
+    if st != 0:
+        raise RuntimeError(f"backward failed: {cp.status_string(st)}")
+    del gq, gk, gv, dod, bws
+
     # --- unfused path: per-step partials + merge kernel
     op = torch.empty(N, plan.rows, D, dtype=torch.float32, device=dev)
     lp = torch.empty(N, plan.rows, dtype=torch.float32, device=dev)
@@ -389,6 +412,10 @@ def main():
             "permute_ms": perm, "permute_gbs": perm_gbs, "permute_frac_hbm": perm_gbs / float(peaks["hbm_gbs"]),
             "rope_permute_ms": rope, "rope_permute_gbs": rope_gbs,
             "rope_permute_frac_hbm": rope_gbs / float(peaks["hbm_gbs"]),
+            "bwd_ms": bwd, "bwd_tflops_useful": 2.5 * w.flops / (bwd * 1e-3) / 1e12,
+            "bwd_tflops_executed": 3.5 * w.flops / (bwd * 1e-3) / 1e12,
+            "bwd_flops_note": "useful = 2.5x the forward's FLOPs (5 tile products); executed = 3.5x "
+                              "(S and dP recomputed by the dQ kernel, no atomics)",
             "partials_ms": part_ms, "merge_ms": merge_ms, "merge_gbs": merge_gbs,
             "merge_frac_hbm": merge_gbs / float(peaks["hbm_gbs"]),
             "unfused_tflops": w.flops / ((part_ms + merge_ms) * 1e-3) / 1e12,
