@@ -19,10 +19,12 @@ Contents:
   * ``rope``       — rotary position embedding at global positions.
   * ``attention_bwd`` — gradients of softmax attention (dQ, dK, dV), by the
     chain rule on the forward's definition.
+  * ``sp_norm``    — reduce-scatter / all-gather over virtual ranks and the
+    LayerNorm + dropout + residual step on sequence shards.
 
 Every function is pinned by ``tests/test_oracle_*.py`` against something other
 than itself (library special cases, closed forms, invariants, hand-derived
 worked examples under ``tests/golden/``). No function here is "parity
 unpinned".
 """
-from . import attention, attention_bwd, layouts, rope, schedule  # noqa: F401
+from . import attention, attention_bwd, layouts, rope, schedule, sp_norm  # noqa: F401
