@@ -327,6 +327,32 @@ def main():
         raise RuntimeError(f"backward failed: {cp.status_string(st)}")
     del gq, gk, gv, dod, bws
 
+    # --- sequence-parallel step after a tensor-parallel region (HBM-bound):
+    # z = dropout(sum of 8 partials) + residual, y = LayerNorm(z); 32768 tokens, H 4096
+    from workloads import make_keep_bits
+    sp_rows, sp_h, sp_n, sp_p = S, 4096, 8, 0.1
+    gsp = torch.Generator().manual_seed(5)
+    sp_parts = torch.randn(sp_n, sp_rows, sp_h, generator=gsp).to(torch.bfloat16).to(dev)
+    sp_res = torch.randn(sp_rows, sp_h, generator=gsp).to(torch.bfloat16).to(dev)
+    sp_gamma = torch.ones(sp_h, device=dev)
+    sp_beta = torch.zeros(sp_h, device=dev)
+    sp_bits = make_keep_bits(sp_rows, sp_h, sp_p, seed=5)[1].to(dev)
+    sp_z = torch.empty(sp_rows, sp_h, dtype=torch.bfloat16, device=dev)
+    sp_y = torch.empty_like(sp_z)
+    sp_ms = []
+    for i in range(7):
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        cp.sp_rs_dropout_add_ln(sp_parts, sp_bits, sp_p, sp_res, sp_gamma, sp_beta, z=sp_z, y=sp_y)
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        if i >= 2:
+            sp_ms.append(a0.elapsed_time(a1))
+    sp_t = statistics.median(sp_ms)
+    sp_bytes = (sp_n + 1 + 2) * sp_rows * sp_h * 2 + sp_rows * sp_h // 8 + 2 * sp_h * 4
+    sp_gbs = sp_bytes / (sp_t * 1e-3) / 1e9
+    del sp_parts, sp_res, sp_bits, sp_z, sp_y
+
     # --- unfused path: per-step partials + merge kernel
     op = torch.empty(N, plan.rows, D, dtype=torch.float32, device=dev)
     lp = torch.empty(N, plan.rows, dtype=torch.float32, device=dev)
@@ -416,6 +442,8 @@ def main():
             "bwd_tflops_executed": 3.5 * w.flops / (bwd * 1e-3) / 1e12,
             "bwd_flops_note": "useful = 2.5x the forward's FLOPs (5 tile products); executed = 3.5x "
                               "(S and dP recomputed by the dQ kernel, no atomics)",
+            "sp_step_ms": sp_t, "sp_step_gbs": sp_gbs, "sp_step_frac_hbm": sp_gbs / float(peaks["hbm_gbs"]),
+            "sp_step_shape": "8 partials x 32768 tokens x H 4096 bf16, dropout 0.1, residual, LayerNorm",
             "partials_ms": part_ms, "merge_ms": merge_ms, "merge_gbs": merge_gbs,
             "merge_frac_hbm": merge_gbs / float(peaks["hbm_gbs"]),
             "unfused_tflops": w.flops / ((part_ms + merge_ms) * 1e-3) / 1e12,

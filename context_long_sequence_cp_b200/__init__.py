@@ -32,6 +32,7 @@ SIGNATURES = {
     "cp_attn_plan_num_items": (_I64, [_P]),
     "cp_attn_plan_cta_loads": (_I64, [_P, _P]),
     "cp_attn_bwd": (_I, [_P] * 12),
+    "cp_sp_rs_dropout_add_ln": (_I, [_P, _I, _I64, _I, _P, ctypes.c_float, _P, _P, _P, ctypes.c_float, _P, _P, _P]),
     "cp_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_P]),
     "cp_attn_plan_bwd_pairs": (_I64, [_P, _P, _P]),
     "cp_attn_workspace_bytes": (_SZ, [_P, _I]),
@@ -235,6 +236,27 @@ def attn_bwd(plan: Plan, q, k, v, o, lse, dout, dq=None, dk=None, dv=None, works
     _check("cp_attn_bwd", lib().cp_attn_bwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
                                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), _stream(stream)))
     return dq, dk, dv
+
+
+def sp_rs_dropout_add_ln(partials, keep_bits=None, p: float = 0.0, residual=None, gamma=None, beta=None,
+                         eps: float = 1e-5, z=None, y=None, want_z=True, want_y=True, stream=None):
+    """``cp_sp_rs_dropout_add_ln``: z = dropout(sum of partials) + residual, y = LayerNorm(z).
+
+    partials: bf16 [nparts, rows, H]; keep_bits: int32/uint32 tensor of packed keep bits."""
+    nparts, rows, H = partials.shape
+    if want_z and z is None:
+        z = torch.empty(rows, H, dtype=torch.bfloat16, device=partials.device)
+    if want_y and gamma is not None and y is None:
+        y = torch.empty(rows, H, dtype=torch.bfloat16, device=partials.device)
+    _check("cp_sp_rs_dropout_add_ln",
+           lib().cp_sp_rs_dropout_add_ln(_ptr(partials), int(nparts), int(rows), int(H),
+                                         _ptr(keep_bits) if keep_bits is not None else None, float(p),
+                                         _ptr(residual) if residual is not None else None,
+                                         _ptr(gamma) if gamma is not None else None,
+                                         _ptr(beta) if beta is not None else None, float(eps),
+                                         _ptr(z) if z is not None else None, _ptr(y) if y is not None else None,
+                                         _stream(stream)))
+    return z, y
 
 
 def layout_index_map(plan: Plan, device="cuda", stream=None):

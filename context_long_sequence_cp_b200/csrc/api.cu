@@ -15,6 +15,7 @@
 
 #include "attn_bwd.h"
 #include "attn_fwd.h"
+#include "sp_norm.h"
 #include "cp_attn.h"
 #include "geometry.h"
 
@@ -651,6 +652,40 @@ int cp_rope_permute(cp_attn_plan_t plan, const void* in, void* out, double base,
   return launch_rope_permute(permute_args(plan, 0, 2), ra, in, out, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? CP_OK
              : CP_ERR_CUDA;
+}
+
+int cp_sp_rs_dropout_add_ln(const void* partials, int nparts, int64_t rows, int H, const uint32_t* keep_bits,
+                            float p, const void* residual, const float* gamma, const float* beta, float eps,
+                            void* z_out, void* y_out, cp_stream_t stream) {
+  if (partials == nullptr || nparts < 1 || rows < 0) return CP_ERR_INVALID_ARG;
+  if (H < 8 || H > 8192 || H % 8 != 0) return CP_ERR_UNSUPPORTED;
+  if (keep_bits != nullptr && !(p >= 0.f && p < 1.f)) return CP_ERR_INVALID_ARG;
+  if ((gamma == nullptr) != (beta == nullptr)) return CP_ERR_INVALID_ARG;
+  if (y_out != nullptr && gamma == nullptr) return CP_ERR_INVALID_ARG;
+  if (z_out == nullptr && y_out == nullptr) return CP_ERR_INVALID_ARG;
+  if (y_out != nullptr && !(eps > 0.f)) return CP_ERR_INVALID_ARG;
+  if (!aligned16(partials) || (residual != nullptr && !aligned16(residual)) || (gamma != nullptr && !aligned16(gamma)) ||
+      (beta != nullptr && !aligned16(beta)) || (z_out != nullptr && !aligned16(z_out)) ||
+      (y_out != nullptr && !aligned16(y_out)) ||
+      (keep_bits != nullptr && (reinterpret_cast<uintptr_t>(keep_bits) & 3u) != 0))
+    return CP_ERR_ALIGNMENT;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) return CP_ERR_CUDA;
+  SpArgs a;
+  a.partials = static_cast<const __nv_bfloat16*>(partials);
+  a.nparts = nparts;
+  a.part_stride = rows * H;
+  a.keep = keep_bits;
+  a.inv_keep = keep_bits != nullptr ? 1.f / (1.f - p) : 1.f;
+  a.residual = static_cast<const __nv_bfloat16*>(residual);
+  a.gamma = gamma;
+  a.beta = beta;
+  a.eps = eps;
+  a.z = static_cast<__nv_bfloat16*>(z_out);
+  a.y = static_cast<__nv_bfloat16*>(y_out);
+  a.rows = rows;
+  a.H = H;
+  return launch_sp_rs_dropout_add_ln(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
 int64_t cp_layout_index_map_len(cp_attn_plan_t plan) {

@@ -189,6 +189,35 @@ CP_API int cp_attn_bwd(cp_attn_plan_t plan, const void* q, const void* k, const 
                        const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
                        cp_stream_t stream);
 
+/*
+ * The sequence-parallel step after a tensor-parallel region (Megatron-style
+ * sequence parallelism), for N virtual ranks on one GPU. Page "序列并行：超长序列
+ * 训练" (guijiagi.com), the MegatronSP example: a reduce-scatter along the sequence
+ * returns each rank its shard of the summed partial outputs, dropout is applied
+ * and the residual added locally, LayerNorm is per token (no communication);
+ * the 5688vip.com page's sequence_parallel_ln_dropout fixes the LayerNorm
+ * (population variance, eps inside the square root, gamma * x_norm + beta) and
+ * training-mode dropout (kept values divided by 1 - p). One fused pass:
+ *   z = keep ? (sum_r partials[r]) / (1 - p) : 0  (+ residual),   y = LayerNorm(z).
+ * On one GPU the ranks' shards are the contiguous row chunks of one buffer, so
+ * the all-gather of the shards is the buffer itself.
+ *
+ * partials: bf16 [nparts][rows][H] (rank r's partial sum at offset r*rows*H);
+ * keep_bits: dropout keep mask, ceil(rows*H/32) uint32 words, bit (i % 32) of
+ *   word i / 32 for flat element i = row*H + h (a host-generated random draw), or
+ *   NULL for no dropout;
+ *   p: the drop rate, 0 <= p < 1;
+ * residual: bf16 [rows][H] or NULL; gamma, beta: fp32 [H], both or neither;
+ *   eps > 0 when y_out is written;
+ * z_out, y_out: bf16 [rows][H] outputs, either may be NULL (not both; y_out needs
+ *   gamma). All device memory, caller-owned, 16-byte aligned (keep_bits 4-byte).
+ * 8 <= H <= 8192, H % 8 == 0 (CP_ERR_UNSUPPORTED otherwise); bad arguments give
+ * CP_ERR_INVALID_ARG, misalignment CP_ERR_ALIGNMENT. Enqueued on `stream`.
+ */
+CP_API int cp_sp_rs_dropout_add_ln(const void* partials, int nparts, int64_t rows, int H, const uint32_t* keep_bits,
+                                   float p, const void* residual, const float* gamma, const float* beta, float eps,
+                                   void* z_out, void* y_out, cp_stream_t stream);
+
 /* Workspace bytes of cp_attn_bwd (0 for a Ulysses plan, which has no backward). */
 CP_API size_t cp_attn_bwd_workspace_bytes(cp_attn_plan_t plan);
 

@@ -210,3 +210,22 @@ def test_bwd_argument_validation():
     assert u.bwd_workspace_bytes() == 0
     p.close()
     u.close()
+
+
+def test_sp_rs_dropout_add_ln_argument_validation():
+    L = cp.lib()
+    P = lambda a: ctypes.c_void_p(a)
+    pt, z, y, g, b, kb = P(4096), P(8192), P(12288), P(16384), P(20480), P(24576)
+    f = L.cp_sp_rs_dropout_add_ln
+    assert f(None, 1, 4, 64, None, 0.0, None, None, None, 1e-5, z, None, None) == -1
+    assert f(pt, 0, 4, 64, None, 0.0, None, None, None, 1e-5, z, None, None) == -1      # nparts < 1
+    assert f(pt, 1, 4, 60, None, 0.0, None, None, None, 1e-5, z, None, None) == -2      # H % 8
+    assert f(pt, 1, 4, 16384, None, 0.0, None, None, None, 1e-5, z, None, None) == -2   # H > 8192
+    assert f(pt, 1, 4, 64, kb, 1.0, None, None, None, 1e-5, z, None, None) == -1        # p must be < 1
+    assert f(pt, 1, 4, 64, None, 0.0, None, g, None, 1e-5, z, None, None) == -1        # gamma without beta
+    assert f(pt, 1, 4, 64, None, 0.0, None, None, None, 1e-5, None, y, None) == -1     # y needs gamma
+    assert f(pt, 1, 4, 64, None, 0.0, None, None, None, 1e-5, None, None, None) == -1  # no output
+    assert f(pt, 1, 4, 64, None, 0.0, None, g, b, 0.0, None, y, None) == -1           # eps > 0
+    assert f(P(4100), 1, 4, 64, None, 0.0, None, None, None, 1e-5, z, None, None) == -3
+    assert f(pt, 1, 4, 64, P(24578), 0.1, None, None, None, 1e-5, z, None, None) == -3  # keep bits 4-aligned
+    assert f(pt, 2, 4, 64, kb, 0.1, None, g, b, 1e-5, z, y, None) in (0, -4)           # no device here

@@ -105,6 +105,19 @@ def make_dout(shape, seed):
     return torch.randn(*shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
 
 
+def make_keep_bits(rows: int, H: int, p: float, seed: int):
+    """Dropout keep mask (the random draw of dropout) for rows x H elements: keep
+    where a seeded uniform draw exceeds p, as the 5688vip.com page's dropout does.
+    Returns (keep bool [rows, H], packed int32 [ceil(rows*H/32)]: bit i % 32 of word
+    i/32 holds flat element i; unused bits of the last word are 0)."""
+    g = torch.Generator("cpu")
+    g.manual_seed(2000 + seed)
+    keep = torch.rand(rows, H, generator=g) > p
+    packed = np.packbits(keep.numpy().reshape(-1), bitorder="little")
+    packed = np.concatenate([packed, np.zeros((-len(packed)) % 4, dtype=np.uint8)]).view(np.int32)
+    return keep.numpy(), torch.from_numpy(packed.copy())
+
+
 def sample_rows(w: Workload, n: Optional[int] = None) -> np.ndarray:
     """Sampled query rows (b, h, i) in natural coordinates, int64 [n_rows, 3].
 
