@@ -22,8 +22,10 @@
 //                      MN-major operands (no transpose is materialised).
 //   attn_bwd_q_kernel  one 128-query tile per work item; walks the key tiles it
 //                      sees in ring order. TMEM: S = Q K^T [0,128), dP = dO V^T
-//                      [128,256), dQ [256,256+D); dS (bf16, from TMEM) times K
-//                      (MN-major) accumulates dQ.
+//                      [128,256), dQ [256,256+D), dS double-buffered as bf16 in
+//                      [384,448) and [448,512); dS (from TMEM) times K (MN-major)
+//                      accumulates dQ. S and dP of the next key tile are computed
+//                      while the current dS is formed.
 // The dK/dV and dQ kernels recompute S and dP each (7 tile products per tile
 // pair instead of 5 with an atomic dQ): the price of having no atomics.
 //
@@ -91,6 +93,17 @@ __device__ __forceinline__ void issue_acc(uint32_t tAcc, uint32_t tX, uint32_t y
   for (int kk = KK_BEGIN; kk < KK_END; ++kk) {
     const uint64_t b = smem_desc_sw128(y_addr + kk * 2048, BwdCfg<D>::kBlockBytes, 1024);
     umma_ts_elect(tAcc, tX + half_col(kk), b, BwdCfg<D>::kIdescAcc, (accumulate || kk > KK_BEGIN) ? 1u : 0u);
+  }
+}
+
+// dQ (+)= dS K over the 128 keys of a tile: dS from a TMEM buffer of 64 packed
+// columns (keys 16kk.. at column 8kk), K a 128 x D tile read as an MN-major operand.
+template <int D>
+__device__ __forceinline__ void issue_dq(uint32_t tdQ, uint32_t tBuf, uint32_t k_addr, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t b = smem_desc_sw128(k_addr + kk * 2048, BwdCfg<D>::kBlockBytes, 1024);
+    umma_ts_elect(tdQ, tBuf + kk * 8, b, BwdCfg<D>::kIdescAcc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -218,6 +231,7 @@ struct alignas(1024) QSmem {
   uint64_t q_full, q_empty;
   uint64_t kv_full[BwdCfg<D>::kStages], kv_empty[BwdCfg<D>::kStages];
   uint64_t s_full;
+  uint64_t sdp_free;   // both warpgroups have read S and dP of the current tile
   uint64_t p_full[2];
   uint64_t acc_done;
   uint64_t drain;
@@ -505,6 +519,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(smem_addr(&sm.kv_empty[s]), 1);
     }
     mbar_init(smem_addr(&sm.s_full), 1);
+    mbar_init(smem_addr(&sm.sdp_free), 256);
     mbar_init(smem_addr(&sm.p_full[0]), 128);
     mbar_init(smem_addr(&sm.p_full[1]), 128);
     mbar_init(smem_addr(&sm.acc_done), 1);
@@ -578,9 +593,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t tS = tbase, tP2 = tbase + 128, tdQ = tbase + 256;
+    // Per key tile e: S(e), dP(e) as soon as the elementwise warps have read
+    // S(e-1), dP(e-1) (sdp_free); then dQ += dS(e-1) K(e-1) once dS(e-1) is in
+    // its buffer (p_full). dS is double-buffered in TMEM columns [384, 512), so
+    // the tensor core computes the next scores while the current dS is formed.
+    const uint32_t tS = tbase, tP2 = tbase + 128, tdQ = tbase + 256, tdS = tbase + 384;
     const uint32_t q_addr = smem_addr(sm.q), do_addr = smem_addr(sm.dout);
-    int q_iter = 0, kv_idx = 0, p_cnt = 0;
+    int q_iter = 0, kv_idx = 0, p_cnt = 0, f_cnt = 0;
+    int tiles = 0;   // tiles issued by this CTA so far (across items)
     bool ok = true, issued = false;
     for (int it = __ldg(p.cta_begin + blockIdx.x); it < it_end && ok; ++it) {
       const WorkItem w = p.items[it];
@@ -593,37 +613,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ++q_iter;
       tc_fence_after();
       bool acc = false;
+      int prev_st = 0;
       for (int e = e_begin; e < e_end; ++e) {
+        const int nt = e - e_begin;
         const int st = kv_idx % C::kStages;
         ok = mbar_wait(smem_addr(&sm.kv_full[st]), (kv_idx / C::kStages) & 1, ctl);
+        // S and dP of the previous tile (of this or the previous item) are read.
+        if (ok && tiles > 0) ok = mbar_wait(smem_addr(&sm.sdp_free), f_cnt & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++kv_idx;
+        if (tiles > 0) ++f_cnt;
+        ++tiles;
         tc_fence_after();
-        const uint32_t k_addr = smem_addr(sm.k[st]), v_addr = smem_addr(sm.v[st]);
-        issue_nt<D>(tS, q_addr, k_addr);     // S = Q K^T
-        issue_nt<D>(tP2, do_addr, v_addr);   // dP = dO V^T
-        umma_commit_elect(smem_addr(&sm.s_full));
+        issue_nt<D>(tS, q_addr, smem_addr(sm.k[st]));      // S = Q K^T
+        issue_nt<D>(tP2, do_addr, smem_addr(sm.v[st]));    // dP = dO V^T
         issued = true;
-        ok = mbar_wait(smem_addr(&sm.p_full[0]), p_cnt & 1, ctl);
-        if (ok && !acc) ok = mbar_wait(smem_addr(&sm.p_full[1]), p_cnt & 1, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        issue_acc<D, 0, 4>(tdQ, tS, k_addr, acc);   // dQ += dS[:, 0:64] K[0:64]
-        if (acc) {
-          ok = mbar_wait(smem_addr(&sm.p_full[1]), p_cnt & 1, ctl);
+        if (nt > 0) {
+          // dS(e-1) of both warpgroups; waited before s_full(e) is committed, so
+          // no warpgroup can arrive for tile e while this wait is pending.
+          ok = mbar_wait(smem_addr(&sm.p_full[0]), p_cnt & 1, ctl);
+          if (ok) ok = mbar_wait(smem_addr(&sm.p_full[1]), p_cnt & 1, ctl);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
+          ++p_cnt;
           tc_fence_after();
+          umma_commit_elect(smem_addr(&sm.s_full));
+          issue_dq<D>(tdQ, tdS + ((nt - 1) & 1) * 64, smem_addr(sm.k[prev_st]), acc);
+          acc = true;
+          umma_commit_elect(smem_addr(&sm.kv_empty[prev_st]));
+        } else {
+          umma_commit_elect(smem_addr(&sm.s_full));
         }
-        issue_acc<D, 4, 8>(tdQ, tS, k_addr, true);
-        ++p_cnt;
-        acc = true;
-        umma_commit_elect(smem_addr(&sm.kv_empty[st]));
+        prev_st = st;
       }
       if (!ok) break;
-      if (e_begin < e_end) umma_commit_elect(smem_addr(&sm.acc_done));
+      if (e_end > e_begin) {
+        ok = mbar_wait(smem_addr(&sm.p_full[0]), p_cnt & 1, ctl);
+        if (ok) ok = mbar_wait(smem_addr(&sm.p_full[1]), p_cnt & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++p_cnt;
+        tc_fence_after();
+        issue_dq<D>(tdQ, tdS + ((e_end - e_begin - 1) & 1) * 64, smem_addr(sm.k[prev_st]), acc);
+        umma_commit_elect(smem_addr(&sm.kv_empty[prev_st]));
+        umma_commit_elect(smem_addr(&sm.acc_done));
+      }
       umma_commit_elect(smem_addr(&sm.q_empty));
     }
     if (issued) {
@@ -636,7 +671,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int quad = warp & 3;
     const int row = quad * 32 + lane;   // query row of the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tS = tbase + lane_off, tP2 = tS + 128, tdQ = tS + 256;
+    const uint32_t tS = tbase + lane_off, tP2 = tS + 128, tdQ = tS + 256, tdS = tS + 384;
     const float sl2 = p.scale_log2;
     int s_cnt = 0, acc_cnt = 0;
     bool ok = true;
@@ -664,23 +699,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // within a rank).
         int lim = kTile;
         if (entry_c0(ent) == kMasked) lim = valid ? column_limit(g, entry_rank(ent), entry_tile(ent) * kTile, gq) : 0;
+        // Read this warpgroup's 64 columns of S and dP, then release them to the
+        // next tile's products before computing dS.
+        uint32_t sa[2][32], da[2][32];
+        tmem_ld32x2(tS + wg * 64, tP2 + wg * 64, sa[0], da[0]);
+        tmem_ld32x2(tS + wg * 64 + 32, tP2 + wg * 64 + 32, sa[1], da[1]);
+        tc_fence_before();
+        mbar_arrive(smem_addr(&sm.sdp_free));
+        const uint32_t tbuf = tdS + (ntile & 1) * 64 + wg * 32;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int col0 = wg * 64 + cc * 32;
-          uint32_t sa[32], da[32];
-          tmem_ld32x2(tS + col0, tP2 + col0, sa, da);
           uint32_t dk[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int c = col0 + 2 * j;
             const bool a0 = c < lim, a1 = c + 1 < lim;
-            const float p0 = a0 ? ex2_approx(__uint_as_float(sa[2 * j]) * sl2 - lse2) : 0.f;
-            const float p1 = a1 ? ex2_approx(__uint_as_float(sa[2 * j + 1]) * sl2 - lse2) : 0.f;
-            const float d0 = a0 ? p0 * (__uint_as_float(da[2 * j]) - drow) : 0.f;
-            const float d1 = a1 ? p1 * (__uint_as_float(da[2 * j + 1]) - drow) : 0.f;
+            const float p0 = a0 ? ex2_approx(__uint_as_float(sa[cc][2 * j]) * sl2 - lse2) : 0.f;
+            const float p1 = a1 ? ex2_approx(__uint_as_float(sa[cc][2 * j + 1]) * sl2 - lse2) : 0.f;
+            const float d0 = a0 ? p0 * (__uint_as_float(da[cc][2 * j]) - drow) : 0.f;
+            const float d1 = a1 ? p1 * (__uint_as_float(da[cc][2 * j + 1]) - drow) : 0.f;
             dk[j] = pack_bf16x2(d0, d1);
           }
-          tmem_st16(tS + wg * 64 + cc * 16, dk);
+          tmem_st16(tbuf + cc * 16, dk);
         }
         tmem_st_wait();
         tc_fence_before();
