@@ -14,12 +14,13 @@
 //                      [NR*B][Hh][T] so that a query tile's 128 values are
 //                      contiguous (one bulk copy).
 //   attn_bwd_kv_kernel one 128-key tile per work item; walks the query tiles
-//                      that see it. TMEM (512 columns): S^T = K Q^T [0,128),
-//                      dP^T = V dO^T [128,256), dV [256,256+D), dK [256+D,256+2D).
-//                      Keys are TMEM lanes, so P^T and dS^T are written back as
-//                      bf16 over their own fp32 columns and feed dV += P^T dO and
+//                      that see it. TMEM (512 columns): region A [0,128) takes
+//                      S^T = K Q^T and then dP^T = V dO^T of the same tile,
+//                      region B [128,256) the bf16 P^T and dS^T, then dV and dK.
+//                      Keys are TMEM lanes, so P^T and dS^T feed dV += P^T dO and
 //                      dK += dS^T Q straight from TMEM; dO and Q are read as
-//                      MN-major operands (no transpose is materialised).
+//                      MN-major operands (no transpose is materialised). The next
+//                      tile's S^T runs while the current P^T/dS^T are formed.
 //   attn_bwd_q_kernel  one 128-query tile per work item; walks the key tiles it
 //                      sees in ring order. TMEM: S = Q K^T [0,128), dP = dO V^T
 //                      [128,256), dQ [256,256+D), dS double-buffered as bf16 in
@@ -214,8 +215,12 @@ struct alignas(1024) KvSmem {
   float dvec[BwdCfg<D>::kStages][kTile];
   uint64_t kv_full, kv_empty;
   uint64_t qd_full[BwdCfg<D>::kStages], qd_empty[BwdCfg<D>::kStages];
-  uint64_t s_full;
-  uint64_t p_full[2];   // [warpgroup]: its half of P^T and dS^T is in TMEM
+  uint64_t s_full;      // S^T of the current tile is in region A
+  uint64_t s_free;      // both warpgroups have read it (256 arrivals)
+  uint64_t dp_full;     // dP^T of the current tile is in region A
+  uint64_t a_free;      // both warpgroups have read it (256 arrivals)
+  uint64_t b_free;      // the products of the previous tile have read region B
+  uint64_t p_full[2];   // [warpgroup]: its half of P^T and dS^T is in region B
   uint64_t acc_done;
   uint64_t drain;
   WaitBlock wblk;
@@ -265,6 +270,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(smem_addr(&sm.qd_empty[s]), 1);
     }
     mbar_init(smem_addr(&sm.s_full), 1);
+    mbar_init(smem_addr(&sm.s_free), 256);
+    mbar_init(smem_addr(&sm.dp_full), 1);
+    mbar_init(smem_addr(&sm.a_free), 256);
+    mbar_init(smem_addr(&sm.b_free), 1);
     mbar_init(smem_addr(&sm.p_full[0]), 128);
     mbar_init(smem_addr(&sm.p_full[1]), 128);
     mbar_init(smem_addr(&sm.acc_done), 1);
@@ -343,9 +352,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t tS = tbase, tP2 = tbase + 128, tdV = tbase + 256, tdK = tbase + 256 + D;
+    // TMEM: region A [0,128) holds S^T(e) and then dP^T(e) (fp32), region B
+    // [128,256) holds P^T(e) at [128,192) and dS^T(e) at [192,256) (bf16), then dV
+    // and dK. Per query tile e the tensor core runs S^T(e), dV/dK(e-1), dP^T(e):
+    // S^T(e) once region A is free (the warpgroups have read dP^T(e-1)), dP^T(e)
+    // once they have read S^T(e), the products of tile e-1 once its P^T and dS^T
+    // are in region B; the warpgroups fill region B only after the products of
+    // the tile before have read it (b_free).
+    const uint32_t tA = tbase, tB = tbase + 128, tdV = tbase + 256, tdK = tbase + 256 + D;
     const uint32_t k_addr = smem_addr(sm.k), v_addr = smem_addr(sm.v);
-    int kv_iter = 0, qd_idx = 0, p_cnt = 0;
+    int kv_iter = 0, qd_idx = 0, p_cnt = 0, a_cnt = 0, sf_cnt = 0;
+    int tiles = 0;   // tiles of this CTA so far (across items)
     bool ok = true, issued = false;
     for (int it = __ldg(p.cta_begin + blockIdx.x); it < it_end && ok; ++it) {
       const WorkItem w = p.items[it];
@@ -358,43 +375,62 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ++kv_iter;
       tc_fence_after();
       bool acc = false;
+      int prev_st = 0;
       for (int e = e_begin; e < e_end; ++e) {
+        const int nt = e - e_begin;
         const int st = qd_idx % C::kStages;
         ok = mbar_wait(smem_addr(&sm.qd_full[st]), (qd_idx / C::kStages) & 1, ctl);
+        if (ok && tiles > 0) ok = mbar_wait(smem_addr(&sm.a_free), a_cnt & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++qd_idx;
+        if (tiles > 0) ++a_cnt;
+        ++tiles;
         tc_fence_after();
         const uint32_t q_addr = smem_addr(sm.q[st]), do_addr = smem_addr(sm.dout[st]);
-        // S^T and dP^T overwrite the bf16 halves of the previous tile only after
-        // the products that read them (issued earlier, tensor-core order).
-        issue_nt<D>(tS, k_addr, q_addr);     // S^T = K Q^T
-        issue_nt<D>(tP2, v_addr, do_addr);   // dP^T = V dO^T
+        issue_nt<D>(tA, k_addr, q_addr);   // S^T(e) = K Q^T
         umma_commit_elect(smem_addr(&sm.s_full));
         issued = true;
-        // The first products of an item overwrite dV and dK, which both
-        // warpgroups read in the previous item's epilogue: wait for both.
-        ok = mbar_wait(smem_addr(&sm.p_full[0]), p_cnt & 1, ctl);
-        if (ok && !acc) ok = mbar_wait(smem_addr(&sm.p_full[1]), p_cnt & 1, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        issue_acc<D, 0, 4>(tdV, tS, do_addr, acc);    // dV += P^T[:, 0:64] dO[0:64]
-        issue_acc<D, 0, 4>(tdK, tP2, q_addr, acc);    // dK += dS^T[:, 0:64] Q[0:64]
-        if (acc) {
-          ok = mbar_wait(smem_addr(&sm.p_full[1]), p_cnt & 1, ctl);
+        if (nt > 0) {
+          // Products of tile e-1 (both warpgroups' halves of P^T and dS^T). The
+          // first of an item overwrites dV and dK, which the previous item's
+          // epilogue read before these halves were stored.
+          ok = mbar_wait(smem_addr(&sm.p_full[0]), p_cnt & 1, ctl);
+          if (ok) ok = mbar_wait(smem_addr(&sm.p_full[1]), p_cnt & 1, ctl);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
+          ++p_cnt;
           tc_fence_after();
+          const uint32_t pq = smem_addr(sm.q[prev_st]), pd = smem_addr(sm.dout[prev_st]);
+          issue_dq<D>(tdV, tB, pd, acc);        // dV += P^T(e-1) dO(e-1)
+          issue_dq<D>(tdK, tB + 64, pq, acc);   // dK += dS^T(e-1) Q(e-1)
+          acc = true;
+          umma_commit_elect(smem_addr(&sm.b_free));
+          umma_commit_elect(smem_addr(&sm.qd_empty[prev_st]));
         }
-        issue_acc<D, 4, 8>(tdV, tS, do_addr, true);
-        issue_acc<D, 4, 8>(tdK, tP2, q_addr, true);
-        ++p_cnt;
-        acc = true;
-        umma_commit_elect(smem_addr(&sm.qd_empty[st]));
+        ok = mbar_wait(smem_addr(&sm.s_free), sf_cnt & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++sf_cnt;
+        tc_fence_after();
+        issue_nt<D>(tA, v_addr, do_addr);   // dP^T(e) = V dO^T, over S^T(e) once read
+        umma_commit_elect(smem_addr(&sm.dp_full));
+        prev_st = st;
       }
       if (!ok) break;
-      if (e_begin < e_end) umma_commit_elect(smem_addr(&sm.acc_done));
+      if (e_end > e_begin) {
+        ok = mbar_wait(smem_addr(&sm.p_full[0]), p_cnt & 1, ctl);
+        if (ok) ok = mbar_wait(smem_addr(&sm.p_full[1]), p_cnt & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++p_cnt;
+        tc_fence_after();
+        issue_dq<D>(tdV, tB, smem_addr(sm.dout[prev_st]), acc);
+        issue_dq<D>(tdK, tB + 64, smem_addr(sm.q[prev_st]), acc);
+        umma_commit_elect(smem_addr(&sm.b_free));
+        umma_commit_elect(smem_addr(&sm.qd_empty[prev_st]));
+        umma_commit_elect(smem_addr(&sm.acc_done));
+      }
       umma_commit_elect(smem_addr(&sm.kv_empty));
     }
     if (issued) {
@@ -407,9 +443,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int quad = warp & 3;
     const int row = quad * 32 + lane;   // key row of the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tS = tbase + lane_off, tP2 = tS + 128, tdV = tS + 256, tdK = tS + 256 + D;
+    const uint32_t tA = tbase + lane_off, tB = tA + 128, tdV = tA + 256, tdK = tA + 256 + D;
     const float sl2 = p.scale_log2;
-    int s_cnt = 0, acc_cnt = 0, qd_idx = 0;
+    int s_cnt = 0, d_cnt = 0, b_cnt = 0, acc_cnt = 0, qd_idx = 0;
+    int tiles = 0;
     bool ok = true;
     for (int it = __ldg(p.cta_begin + blockIdx.x); it < it_end && ok; ++it) {
       const WorkItem w = p.items[it];
@@ -423,9 +460,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int e = e_begin; e < e_end; ++e) {
         const uint32_t ent = __ldg(p.entries + e);
         const int st = qd_idx % C::kStages;
-        // This stage's lse2 / dvec vectors come by bulk copy: wait for them
-        // directly (the phase is complete by now and cannot move on before this
-        // warpgroup's p_full of the tile).
+        // The stage's lse2 / dvec vectors come by bulk copy: wait for them directly.
         ok = mbar_wait(smem_addr(&sm.qd_full[st]), (qd_idx / C::kStages) & 1, ctl);
         ++qd_idx;
         if (ok) ok = mbar_wait(smem_addr(&sm.s_full), s_cnt & 1, ctl);
@@ -433,8 +468,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
-        // Allowed query columns [lo, hi) of this key row: queries at or after the
-        // key in global position, inside the rank's T tokens.
+        // Allowed query columns [lo, hi) of this key row.
         int lo = 0, hi = kTile;
         if (entry_c0(ent) == kMasked) {
           const int rq = entry_rank(ent), q0 = entry_tile(ent) * kTile;
@@ -444,28 +478,60 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         const float* l2 = sm.lse2[st];
         const float* dr = sm.dvec[st];
-#pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          const int col0 = wg * 64 + cc * 32;
-          uint32_t sa[32], da[32];
-          tmem_ld32x2(tS + col0, tP2 + col0, sa, da);
-          uint32_t pk[16], dk[16];
+        // P^T of this warpgroup's 64 query columns from S^T, packed to bf16 (the
+        // values dV's product uses; dS^T below is formed from the same values).
+        uint32_t pk[32];
+        {
+          uint32_t sa[32], sb[32];
+          tmem_ld32x2(tA + wg * 64, tA + wg * 64 + 32, sa, sb);
+          tc_fence_before();
+          mbar_arrive(smem_addr(&sm.s_free));   // region A may take dP^T
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int c = col0 + 2 * j;
-            const float2 lv = *reinterpret_cast<const float2*>(l2 + c);
-            const float2 dv = *reinterpret_cast<const float2*>(dr + c);
-            const bool a0 = c >= lo && c < hi, a1 = c + 1 >= lo && c + 1 < hi;
-            const float p0 = a0 ? ex2_approx(__uint_as_float(sa[2 * j]) * sl2 - lv.x) : 0.f;
-            const float p1 = a1 ? ex2_approx(__uint_as_float(sa[2 * j + 1]) * sl2 - lv.y) : 0.f;
-            const float d0 = a0 ? p0 * (__uint_as_float(da[2 * j]) - dv.x) : 0.f;
-            const float d1 = a1 ? p1 * (__uint_as_float(da[2 * j + 1]) - dv.y) : 0.f;
+            const int c = wg * 64 + 2 * j;
+            const float p0 = (c >= lo && c < hi) ? ex2_approx(__uint_as_float(sa[2 * j]) * sl2 - l2[c]) : 0.f;
+            const float p1 = (c + 1 >= lo && c + 1 < hi) ? ex2_approx(__uint_as_float(sa[2 * j + 1]) * sl2 - l2[c + 1]) : 0.f;
+            const float p2 = (c + 32 >= lo && c + 32 < hi) ? ex2_approx(__uint_as_float(sb[2 * j]) * sl2 - l2[c + 32]) : 0.f;
+            const float p3 = (c + 33 >= lo && c + 33 < hi) ? ex2_approx(__uint_as_float(sb[2 * j + 1]) * sl2 - l2[c + 33]) : 0.f;
             pk[j] = pack_bf16x2(p0, p1);
-            dk[j] = pack_bf16x2(d0, d1);
+            pk[16 + j] = pack_bf16x2(p2, p3);
           }
-          tmem_st16(tS + wg * 64 + cc * 16, pk);
-          tmem_st16(tP2 + wg * 64 + cc * 16, dk);
         }
+        ok = mbar_wait(smem_addr(&sm.dp_full), d_cnt & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++d_cnt;
+        tc_fence_after();
+        uint32_t dk[32];
+        {
+          uint32_t da[32], db[32];
+          tmem_ld32x2(tA + wg * 64, tA + wg * 64 + 32, da, db);
+          tc_fence_before();
+          mbar_arrive(smem_addr(&sm.a_free));   // region A may take the next S^T
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int c = wg * 64 + 2 * j;
+            const float d0 = __uint_as_float(pk[j] << 16) * (__uint_as_float(da[2 * j]) - dr[c]);
+            const float d1 = __uint_as_float(pk[j] & 0xffff0000u) * (__uint_as_float(da[2 * j + 1]) - dr[c + 1]);
+            const float d2 = __uint_as_float(pk[16 + j] << 16) * (__uint_as_float(db[2 * j]) - dr[c + 32]);
+            const float d3 = __uint_as_float(pk[16 + j] & 0xffff0000u) * (__uint_as_float(db[2 * j + 1]) - dr[c + 33]);
+            dk[j] = pack_bf16x2(d0, d1);
+            dk[16 + j] = pack_bf16x2(d2, d3);
+          }
+        }
+        // Region B is free once the products of the previous tile have read it.
+        if (tiles > 0) {
+          ok = mbar_wait(smem_addr(&sm.b_free), b_cnt & 1, ctl);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ++b_cnt;
+          tc_fence_after();
+        }
+        ++tiles;
+        tmem_st16(tB + wg * 32, pk);
+        tmem_st16(tB + wg * 32 + 16, pk + 16);
+        tmem_st16(tB + 64 + wg * 32, dk);
+        tmem_st16(tB + 64 + wg * 32 + 16, dk + 16);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(smem_addr(&sm.p_full[wg]));
