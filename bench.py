@@ -183,7 +183,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["attn", "merge", "permute"], default=None,
+    ap.add_argument("--profile", choices=["attn", "merge", "permute", "bwd"], default=None,
                     help="only launch one kernel warmup+steps times (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -238,8 +238,17 @@ def main():
             cp.attn_fwd_partials(plan, qz, kz, vz, o_parts=op, lse_parts=lp)
             om = torch.empty(plan.rows, D, dtype=torch.bfloat16, device=dev)
             lm = torch.empty(plan.rows, dtype=torch.float32, device=dev)
+        if args.profile == "bwd":
+            from workloads import make_dout
+            dod = torch.empty_like(qz)
+            cp.layout_permute(plan, make_dout(q_h.shape, w.seed).to(dev), 0, out=dod)
+            cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=lse)
+            gq, gk, gv = (torch.empty_like(qz) for _ in range(3))
+            bws = torch.empty(plan.bwd_workspace_bytes(), dtype=torch.uint8, device=dev)
         for _ in range(args.warmup + args.steps):
-            if args.profile == "attn":
+            if args.profile == "bwd":
+                cp.attn_bwd(plan, qz, kz, vz, oz, lse, dod, gq, gk, gv, bws)
+            elif args.profile == "attn":
                 cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=lse)
             elif args.profile == "merge":
                 cp.merge_partials(op, lp, o_out=om, lse_out=lm)
