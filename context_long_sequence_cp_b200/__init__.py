@@ -47,6 +47,16 @@ SIGNATURES = {
     "cp_status_string": (ctypes.c_char_p, [_I]),
     "cp_debug_wait_timeout_probe": (_I, [_P, _I, _P]),
     "cp_attn_fwd_ulysses_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P]),
+    "cp_attn_fwd_ring_step": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "cp_attn_ring_prepare": (_I, [_P, _I]),
+    "cp_attn_ring_schedule": (_I64, [_P, _I, _I, _P, _P]),
+    "cp_ring_buffer_alloc": (_I, [_SZ, ctypes.POINTER(_P)]),
+    "cp_ring_buffer_free": (_I, [_P]),
+    "cp_ipc_handle_bytes": (_I, []),
+    "cp_ipc_get_handle": (_I, [_P, _P]),
+    "cp_ipc_open_handle": (_I, [_P, ctypes.POINTER(_P)]),
+    "cp_ipc_close_handle": (_I, [_P]),
+    "cp_copy_async": (_I, [_P, _P, _SZ, _P]),
 }
 
 # Size of the library's fixed device scratch used by the no-alloc Ulysses
@@ -152,6 +162,24 @@ class Plan:
         lib().cp_attn_plan_cta_loads(self._h, ctypes.cast(arr, ctypes.c_void_p))
         return list(arr)[:n]
 
+    def ring_prepare(self, rank: int):
+        """Build (and upload) the per-step schedules of one rank's ring steps."""
+        _check("cp_attn_ring_prepare", lib().cp_attn_ring_prepare(self._h, int(rank)))
+
+    def ring_schedule(self, rank: int, step: int):
+        """Schedule of one rank's ring step: (items as rows of (row block, head,
+        query-tile pair, key tiles, CTA) in run order, per-CTA modelled loads)."""
+        n = int(lib().cp_attn_ring_schedule(self._h, int(rank), int(step), None, None))
+        if n < 0:
+            raise CpAttnError("cp_attn_ring_schedule", n)
+        items = (ctypes.c_int32 * (5 * n))()
+        loads = (ctypes.c_int64 * max(n, 1))()
+        lib().cp_attn_ring_schedule(self._h, int(rank), int(step), ctypes.cast(items, ctypes.c_void_p),
+                                    ctypes.cast(loads, ctypes.c_void_p))
+        rows = [tuple(items[5 * i:5 * i + 5]) for i in range(n)]
+        n_cta = max(r[4] for r in rows) + 1 if rows else 0
+        return rows, list(loads)[:n_cta]
+
     def workspace_bytes(self, with_partials: bool = False) -> int:
         return int(lib().cp_attn_workspace_bytes(self._h, int(with_partials)))
 
@@ -187,6 +215,94 @@ def attn_fwd_partials(plan: Plan, q, k, v, o_parts=None, lse_parts=None, stream=
                                                               _ptr(o_parts), _ptr(lse_parts), None,
                                                               _stream(stream)))
     return o_parts, lse_parts
+
+
+def attn_fwd_ring_step(plan: Plan, rank: int, step: int, q, k, v, o_part=None, lse_part=None, stream=None):
+    """``cp_attn_fwd_ring_step``: rank ``rank``'s partial against the key/value block
+    of rank (rank + step) mod N, all buffers rank-local [B, S/N, H, D].
+    Returns (o_part fp32 [rows, D], lse_part fp32 [rows]), rows = B*(S/N)*H."""
+    rows = plan.B * (plan.S // plan.N) * plan.H
+    if o_part is None:
+        o_part = torch.empty(rows, plan.D, dtype=torch.float32, device=q.device)
+    if lse_part is None:
+        lse_part = torch.empty(rows, dtype=torch.float32, device=q.device)
+    _check("cp_attn_fwd_ring_step",
+           lib().cp_attn_fwd_ring_step(plan.handle, int(rank), int(step), _ptr(q), _ptr(k), _ptr(v), _ptr(o_part),
+                                       _ptr(lse_part), _stream(stream)))
+    return o_part, lse_part
+
+
+def copy_async(dst_ptr: int, src_ptr: int, nbytes: int, stream=None):
+    """``cp_copy_async``: one device-to-device copy (a peer's memory included)."""
+    _check("cp_copy_async", lib().cp_copy_async(ctypes.c_void_p(int(dst_ptr)), ctypes.c_void_p(int(src_ptr)),
+                                                 int(nbytes), _stream(stream)))
+
+
+class DeviceBuffer:
+    """Device memory from ``cp_ring_buffer_alloc`` (shareable with other processes
+    through CUDA IPC), viewable as a torch tensor without a copy."""
+
+    def __init__(self, nbytes: int):
+        p = ctypes.c_void_p()
+        _check("cp_ring_buffer_alloc", lib().cp_ring_buffer_alloc(int(nbytes), ctypes.byref(p)))
+        self.ptr, self.nbytes = int(p.value), int(nbytes)
+
+    def ipc_handle(self) -> bytes:
+        buf = ctypes.create_string_buffer(int(lib().cp_ipc_handle_bytes()))
+        _check("cp_ipc_get_handle", lib().cp_ipc_get_handle(ctypes.c_void_p(self.ptr), buf))
+        return buf.raw
+
+    def view(self, shape, dtype=torch.bfloat16, offset_bytes: int = 0, device=None):
+        return _device_view(self.ptr + offset_bytes, shape, dtype, device)
+
+    def close(self):
+        if getattr(self, "ptr", 0):
+            lib().cp_ring_buffer_free(ctypes.c_void_p(self.ptr))
+            self.ptr = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class PeerBuffer:
+    """Another process's ``DeviceBuffer`` mapped into this one (``cp_ipc_open_handle``)."""
+
+    def __init__(self, handle: bytes, nbytes: int):
+        p = ctypes.c_void_p()
+        _check("cp_ipc_open_handle", lib().cp_ipc_open_handle(ctypes.c_char_p(handle), ctypes.byref(p)))
+        self.ptr, self.nbytes = int(p.value), int(nbytes)
+
+    def close(self):
+        if getattr(self, "ptr", 0):
+            lib().cp_ipc_close_handle(ctypes.c_void_p(self.ptr))
+            self.ptr = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+_TYPESTR = {torch.bfloat16: "<V2", torch.float32: "<f4", torch.int32: "<i4", torch.uint8: "|u1"}
+
+
+class _CudaArray:
+    def __init__(self, ptr, shape, typestr):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (int(ptr), False),
+                                         "version": 3, "strides": None}
+
+
+def _device_view(ptr: int, shape, dtype, device=None):
+    """A torch tensor over device memory at ``ptr`` (no copy; the memory's owner
+    must outlive it)."""
+    if dtype == torch.bfloat16:
+        t = torch.as_tensor(_CudaArray(ptr, shape, "<i2"), device=device)
+        return t.view(torch.bfloat16)
+    return torch.as_tensor(_CudaArray(ptr, shape, _TYPESTR[dtype]), device=device)
 
 
 def merge_partials(o_parts, lse_parts, o_out=None, lse_out=None, stream=None):

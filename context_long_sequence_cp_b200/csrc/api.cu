@@ -21,6 +21,8 @@
 
 using namespace cpattn;
 
+constexpr int kDefaultSmCountPlan = 148;   // B200; used when no device is visible
+
 struct cp_attn_plan_s {
   int B, H, S, D, N, causal, layout;
   float scale;
@@ -61,12 +63,27 @@ struct cp_attn_plan_s {
   };
   int ntiles = 0;
   BwdSched bwd_kv, bwd_q;
+  // Rank-local ring steps (contiguous and zigzag layouts): for one rank and each
+  // ring step t, that rank's items ordered and assigned to CTAs by their walk at
+  // step t alone. Built for a rank on first use.
+  struct RingRank {
+    bool built = false;
+    int nper = 0;                     // items per step: B * H * query-tile pairs
+    std::vector<WorkItem> items;      // [NR][nper], step t's list at t * nper
+    std::vector<int> cta_begin;       // [NR][sms + 1], step t's at t * (sms + 1)
+    std::vector<int> n_cta;           // [NR]
+    std::vector<int64_t> cta_load;    // [NR][sms]
+    WorkItem* d_items = nullptr;
+    int* d_cta_begin = nullptr;
+  };
+  int sms = kDefaultSmCountPlan;
+  std::vector<RingRank> ring;
 };
 
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per in-kernel wait
-constexpr int kDefaultSmCount = 148;               // B200; used when no device is visible
+constexpr int kDefaultSmCount = kDefaultSmCountPlan;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -89,11 +106,13 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // 4-D view (D, Hh, T, NR*B) of a bf16 tensor stored [NR*B][T][Hh][D]; box of
 // 64 x 1 x 128 x 1 elements (128 B x 128 rows) with the 128-byte swizzle.
-int encode_view(CUtensorMap* map, const void* base, const Geometry& g, int D) {
+// A rank-local buffer holds B row blocks only (row_blocks = B).
+int encode_view(CUtensorMap* map, const void* base, const Geometry& g, int D, int64_t row_blocks = -1) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return CP_ERR_CUDA;
+  if (row_blocks < 0) row_blocks = static_cast<int64_t>(g.NR) * g.B;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(g.Hh),
-                              static_cast<cuuint64_t>(g.T), static_cast<cuuint64_t>(g.NR) * g.B};
+                              static_cast<cuuint64_t>(g.T), static_cast<cuuint64_t>(row_blocks)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(g.Hh) * D * 2,
                                  static_cast<cuuint64_t>(g.T) * g.Hh * D * 2};
   const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kTile), 1};
@@ -249,6 +268,64 @@ int ensure_device(cp_attn_plan_s* p) {
   return CP_ERR_CUDA;
 }
 
+// Schedules of one rank's ring steps: at step t the rank's items (every batch,
+// head and query-tile pair) carry the key tiles of their walk at step t, and are
+// assigned to CTAs by the whole-view list's greedy rule, longest first.
+void build_ring_rank(cp_attn_plan_s* p, int r) {
+  cp_attn_plan_s::RingRank& rr = p->ring[r];
+  const Geometry& g = p->g;
+  const int stride = p->sms + 1;
+  rr.nper = g.B * g.Hh * p->npairs;
+  rr.items.clear();
+  rr.items.reserve(static_cast<size_t>(g.NR) * rr.nper);
+  rr.cta_begin.assign(static_cast<size_t>(g.NR) * stride, 0);
+  rr.cta_load.assign(static_cast<size_t>(g.NR) * p->sms, 0);
+  rr.n_cta.assign(g.NR, 0);
+  for (int t = 0; t < g.NR; ++t) {
+    std::vector<WorkItem> items;
+    items.reserve(rr.nper);
+    for (int b = 0; b < g.B; ++b)
+      for (int qp = 0; qp < p->npairs; ++qp) {
+        const int* off = p->step_off.data() + static_cast<size_t>(r * p->npairs + qp) * (g.NR + 1);
+        const int len = off[t + 1] - off[t];
+        for (int h = 0; h < g.Hh; ++h) items.push_back(WorkItem{r * g.B + b, h, qp, len});
+      }
+    // Longest first: one step has few items per CTA (about 3.5 on 32 heads of
+    // 32k tokens over 8 ranks), and one rank's key/value block stays in L2
+    // whatever the order, so the order serves the balance alone.
+    std::stable_sort(items.begin(), items.end(), [](const WorkItem& a, const WorkItem& b) { return a.cost > b.cost; });
+    std::vector<int64_t> cost(items.size());
+    for (size_t i = 0; i < items.size(); ++i) cost[i] = 2 * static_cast<int64_t>(items[i].cost) + kItemOverheadHalfTiles;
+    std::vector<int> cb;
+    std::vector<int64_t> load;
+    rr.n_cta[t] = assign_greedy(items, cost, p->sms, cb, load);
+    std::copy(cb.begin(), cb.end(), rr.cta_begin.begin() + static_cast<size_t>(t) * stride);
+    std::copy(load.begin(), load.end(), rr.cta_load.begin() + static_cast<size_t>(t) * p->sms);
+    rr.items.insert(rr.items.end(), items.begin(), items.end());
+  }
+  rr.built = true;
+}
+
+void free_ring(cp_attn_plan_s::RingRank& rr) {
+  if (rr.d_items != nullptr) cudaFree(rr.d_items);
+  if (rr.d_cta_begin != nullptr) cudaFree(rr.d_cta_begin);
+  rr.d_items = nullptr;
+  rr.d_cta_begin = nullptr;
+}
+
+int upload_ring_rank(cp_attn_plan_s::RingRank& rr) {
+  if (rr.d_items != nullptr) return CP_OK;
+  const size_t ib = rr.items.size() * sizeof(WorkItem), cb = rr.cta_begin.size() * sizeof(int);
+  const bool ok = cudaMalloc(&rr.d_items, ib) == cudaSuccess && cudaMalloc(&rr.d_cta_begin, cb) == cudaSuccess &&
+                  cudaMemcpy(rr.d_items, rr.items.data(), ib, cudaMemcpyHostToDevice) == cudaSuccess &&
+                  cudaMemcpy(rr.d_cta_begin, rr.cta_begin.data(), cb, cudaMemcpyHostToDevice) == cudaSuccess;
+  if (!ok) {
+    free_ring(rr);
+    return CP_ERR_CUDA;
+  }
+  return CP_OK;
+}
+
 int launch_view(cp_attn_plan_s* p, const Geometry& g, const void* q, const void* k, const void* v, void* o,
                 float* lse, float* o_part, float* lse_part, int t0, int t1, bool partial, cudaStream_t st) {
   FwdLaunch L;
@@ -397,6 +474,8 @@ int cp_attn_plan(cp_attn_plan_t* out, int B, int H, int S, int D, int N, int cau
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess || sms <= 0)
       sms = kDefaultSmCount;
   }
+  p->sms = sms;
+  p->ring.resize(layout == CP_LAYOUT_ULYSSES ? 0 : g.NR);
   schedule_items(p, sms);
   if (layout != CP_LAYOUT_ULYSSES) build_bwd(p, sms);
   if (have_device) {
@@ -443,6 +522,7 @@ int cp_attn_plan_destroy(cp_attn_plan_t plan) {
   if (plan->d_cta_begin != nullptr) cudaFree(plan->d_cta_begin);
   free_bwd(plan->bwd_kv);
   free_bwd(plan->bwd_q);
+  for (auto& rr : plan->ring) free_ring(rr);
   if (plan->d_status != nullptr) cudaFree(plan->d_status);
   if (plan->d_step_off != nullptr) cudaFree(plan->d_step_off);
   if (plan->d_entries != nullptr) cudaFree(plan->d_entries);
@@ -604,6 +684,80 @@ int cp_attn_fwd_partials(cp_attn_plan_t plan, const void* q, const void* k, cons
     if (rc != CP_OK) return rc;
   }
   return CP_OK;
+}
+
+int cp_attn_ring_prepare(cp_attn_plan_t plan, int rank) {
+  if (plan == nullptr) return CP_ERR_INVALID_ARG;
+  if (plan->layout == CP_LAYOUT_ULYSSES) return CP_ERR_UNSUPPORTED;
+  if (rank < 0 || rank >= plan->N) return CP_ERR_INVALID_ARG;
+  cp_attn_plan_s::RingRank& rr = plan->ring[rank];
+  if (!rr.built) build_ring_rank(plan, rank);
+  if (plan->d_items == nullptr) return CP_OK;   // no device: host schedules only
+  return upload_ring_rank(rr);
+}
+
+int64_t cp_attn_ring_schedule(cp_attn_plan_t plan, int rank, int step, int32_t* items, int64_t* cta_loads) {
+  if (plan == nullptr) return CP_ERR_INVALID_ARG;
+  if (plan->layout == CP_LAYOUT_ULYSSES) return CP_ERR_UNSUPPORTED;
+  if (rank < 0 || rank >= plan->N || step < 0 || step >= plan->N) return CP_ERR_INVALID_ARG;
+  cp_attn_plan_s::RingRank& rr = plan->ring[rank];
+  if (!rr.built) build_ring_rank(plan, rank);
+  const int stride = plan->sms + 1;
+  const int* cb = rr.cta_begin.data() + static_cast<size_t>(step) * stride;
+  const WorkItem* it = rr.items.data() + static_cast<size_t>(step) * rr.nper;
+  const int n_cta = rr.n_cta[step];
+  if (items != nullptr)
+    for (int c = 0; c < n_cta; ++c)
+      for (int i = cb[c]; i < cb[c + 1]; ++i) {
+        int32_t* o = items + static_cast<size_t>(i) * 5;
+        o[0] = it[i].rb;
+        o[1] = it[i].h;
+        o[2] = it[i].qp;
+        o[3] = it[i].cost;
+        o[4] = c;
+      }
+  if (cta_loads != nullptr)
+    for (int c = 0; c < n_cta; ++c) cta_loads[c] = rr.cta_load[static_cast<size_t>(step) * plan->sms + c];
+  return rr.nper;
+}
+
+int cp_attn_fwd_ring_step(cp_attn_plan_t plan, int rank, int step, const void* q, const void* k, const void* v,
+                          float* o_part, float* lse_part, cp_stream_t stream) {
+  if (plan == nullptr || q == nullptr || k == nullptr || v == nullptr || o_part == nullptr || lse_part == nullptr)
+    return CP_ERR_INVALID_ARG;
+  if (plan->layout == CP_LAYOUT_ULYSSES) return CP_ERR_UNSUPPORTED;
+  if (rank < 0 || rank >= plan->N || step < 0 || step >= plan->N) return CP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part) || !aligned16(lse_part))
+    return CP_ERR_ALIGNMENT;
+  int rc = ensure_device(plan);
+  if (rc != CP_OK) return rc;
+  if ((rc = cp_attn_ring_prepare(plan, rank)) != CP_OK) return rc;
+  const cp_attn_plan_s::RingRank& rr = plan->ring[rank];
+  const Geometry& g = plan->g;
+  FwdLaunch L;
+  std::memset(&L, 0, sizeof(L));
+  if ((rc = encode_view(&L.tm_q, q, g, plan->D, g.B)) != CP_OK) return rc;
+  if ((rc = encode_view(&L.tm_k, k, g, plan->D, g.B)) != CP_OK) return rc;
+  if ((rc = encode_view(&L.tm_v, v, g, plan->D, g.B)) != CP_OK) return rc;
+  FwdParams& P = L.params;
+  P.g = g;
+  P.t_begin = step;
+  P.t_end = step + 1;
+  P.scale_log2 = plan->scale * 1.4426950408889634f;
+  P.items = rr.d_items + static_cast<size_t>(step) * rr.nper;
+  P.n_items = rr.nper;
+  P.cta_begin = rr.d_cta_begin + static_cast<size_t>(step) * (plan->sms + 1);
+  P.n_cta = rr.n_cta[step];
+  P.step_off = plan->d_step_off;
+  P.entries = plan->d_entries;
+  P.npairs = plan->npairs;
+  P.o_part = o_part;
+  P.lse_part = lse_part;
+  P.q_rb0 = rank * g.B;
+  P.kv_local = 1;
+  P.status = plan->d_status;
+  P.wait_limit_ns = kWaitLimitNs;
+  return launch_attn_fwd(L, plan->D, true, static_cast<cudaStream_t>(stream)) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
 int cp_merge_partials(int num_parts, int64_t rows, int D, const float* o_parts, const float* lse_parts,

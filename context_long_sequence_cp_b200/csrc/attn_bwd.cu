@@ -69,10 +69,6 @@ struct BwdCfg {
   static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, 0, 1);   // A from TMEM, B MN-major
 };
 
-// TMEM column of the bf16 half written for MMA K-step kk (16 columns of the
-// 128-wide tile per step, 8 packed TMEM columns): steps 0-3 at [0,32), 4-7 at [64,96).
-__device__ __forceinline__ uint32_t half_col(int kk) { return kk * 8 + (kk >= 4 ? 32 : 0); }
-
 // C = A B^T over K = D: A and B are 128 x D bf16 tiles, both K-major (the
 // forward's score product form).
 template <int D>
@@ -82,18 +78,6 @@ __device__ __forceinline__ void issue_nt(uint32_t tC, uint32_t a_addr, uint32_t 
     const uint32_t off = (kk >> 2) * BwdCfg<D>::kBlockBytes + (kk & 3) * 32;
     umma_ss_elect(tC, smem_desc_sw128(a_addr + off, 16, 1024), smem_desc_sw128(b_addr + off, 16, 1024),
                   BwdCfg<D>::kIdescS, kk > 0 ? 1u : 0u);
-  }
-}
-
-// Acc (+)= X Y over rows [16*KK_BEGIN, 16*KK_END) of the 128-row tile Y: X from
-// TMEM (bf16, half layout), Y a 128 x D bf16 tile in shared memory read as an
-// MN-major operand (8-row groups 1024 B apart, 64-column blocks kBlockBytes apart).
-template <int D, int KK_BEGIN, int KK_END>
-__device__ __forceinline__ void issue_acc(uint32_t tAcc, uint32_t tX, uint32_t y_addr, bool accumulate) {
-#pragma unroll
-  for (int kk = KK_BEGIN; kk < KK_END; ++kk) {
-    const uint64_t b = smem_desc_sw128(y_addr + kk * 2048, BwdCfg<D>::kBlockBytes, 1024);
-    umma_ts_elect(tAcc, tX + half_col(kk), b, BwdCfg<D>::kIdescAcc, (accumulate || kk > KK_BEGIN) ? 1u : 0u);
   }
 }
 

@@ -246,11 +246,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i)
           for (int blk = 0; blk < C::kBlocks; ++blk)
             tma_load_4d_elect(smem_addr(&sm.q[i][0]) + blk * C::kBlockBytes, &tm_q, qbar, blk * 64, w.h,
-                        q0 + i * kTile, w.rb, pol_q);
+                        q0 + i * kTile, w.rb - p.q_rb0, pol_q);
         ++q_iter;
         for (int e = e_begin; e < e_end && ok; ++e) {
           const uint32_t ent = __ldg(p.entries + e);
-          const int rbk = entry_rank(ent) * g.B + bv;
+          const int rbk = p.kv_local ? bv : entry_rank(ent) * g.B + bv;
           const int k0 = entry_tile(ent) * kTile;
           for (int which = 0; which < 2; ++which) {
             const int stage = kv_idx % C::kStages;
@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const WorkItem w = ld_item_volatile(p.items + it);
       const int bv = w.rb % g.B;
       const int tl = w.qp * kPair + wg * kTile + row;
-      const int64_t row_id = (static_cast<int64_t>(w.rb) * g.T + tl) * g.Hh + w.h;
+      const int64_t row_id = (static_cast<int64_t>(w.rb - p.q_rb0) * g.T + tl) * g.Hh + w.h;
       if (ntile > 0) {
         ok = mbar_wait(smem_addr(&sm.o_done[wg]), od_cnt & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);

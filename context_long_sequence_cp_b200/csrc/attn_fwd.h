@@ -30,6 +30,11 @@ struct FwdParams {
   int64_t lse_S;
   float* o_part;               // partial mode: [rows][D], row = (rb*T + tl)*Hh + h
   float* lse_part;             // partial mode: [rows]
+  // Rank-local buffers (one ring step of one rank): q, o and the partials hold
+  // row blocks from q_rb0 on (0 for the whole view), and with kv_local the k and
+  // v maps hold the key rank's B row blocks only.
+  int q_rb0;
+  int kv_local;
   int* status;                 // device status word (0 = ok)
   uint64_t wait_limit_ns;      // budget of one in-kernel wait
 };

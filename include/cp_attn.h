@@ -165,6 +165,68 @@ CP_API int cp_attn_fwd_partials(cp_attn_plan_t plan, const void* q, const void* 
                          cp_stream_t stream);
 
 /*
+ * One ring step of one rank, on rank-local buffers (contiguous and zigzag
+ * layouts; CP_ERR_UNSUPPORTED for Ulysses). Page "序列与上下文并行", section
+ * "上下文并行：注意力本身切分": rank r holds its own Q/K/V chunk and, at ring step
+ * t, computes the partial attention of its queries against the key/value block
+ * of rank (r+t) mod N, which it has received from the ring; the N partials are
+ * merged by online softmax (cp_merge_partials). Causal masking uses the global
+ * positions of the two ranks' tokens under the plan's layout.
+ *   rank, step : 0 <= rank, step < N
+ *   q          : bf16 [B][S/N][H][D], rank's own chunk (its local tokens in the
+ *                layout's order: zigzag rank r holds chunks r and 2N-1-r), device
+ *   k, v       : bf16 [B][S/N][H][D], the block of rank (rank+step) mod N, device
+ *   o_part     : float32 [B*(S/N)*H][D], row = (b*(S/N) + tl)*H + h, device (written)
+ *   lse_part   : float32 [B*(S/N)*H], same rows, device (written)
+ * O is normalised over the step's keys, lse is natural-log; a row with no
+ * allowed key in the step gets O = 0, lse = -inf. One kernel is enqueued on
+ * `stream`. The first call for a rank builds that rank's per-step schedules and
+ * copies them to the device synchronously (cp_attn_ring_prepare does it ahead of
+ * time, e.g. before a stream capture). Errors: CP_ERR_INVALID_ARG (null pointer,
+ * rank or step out of range), CP_ERR_ALIGNMENT (a pointer not 16-byte aligned),
+ * CP_ERR_CUDA (no device, launch failure); an in-kernel wait that runs out is
+ * reported by cp_attn_check as CP_ERR_TIMEOUT.
+ */
+CP_API int cp_attn_fwd_ring_step(cp_attn_plan_t plan, int rank, int step, const void* q, const void* k,
+                                 const void* v, float* o_part, float* lse_part, cp_stream_t stream);
+
+/* Builds (and, with a device, uploads) the per-step schedules of one rank's ring
+ * steps. Idempotent. Errors: CP_ERR_INVALID_ARG, CP_ERR_UNSUPPORTED (Ulysses),
+ * CP_ERR_CUDA (device allocation). */
+CP_API int cp_attn_ring_prepare(cp_attn_plan_t plan, int rank);
+
+/*
+ * Host-side view of the schedule of one rank's ring step (works without a
+ * device). Returns the number of items n (B*H*query-tile pairs) or a negative
+ * status; when items is not NULL writes n records of five int32 (row block
+ * rank*B + b, head, query-tile pair, executed key tiles of the step, CTA) in
+ * run order; when cta_loads is not NULL writes each CTA's modelled load (as
+ * cp_attn_plan_cta_loads counts it; min(n, SM count) CTAs).
+ */
+CP_API int64_t cp_attn_ring_schedule(cp_attn_plan_t plan, int rank, int step, int32_t* items,
+                                     int64_t* cta_loads);
+
+/*
+ * Plumbing of the multi-GPU ring (one process per GPU). A rank's receive slots
+ * are allocated with cp_ring_buffer_alloc so that the neighbour's process can
+ * map them: cp_ipc_get_handle writes the allocation's handle
+ * (cp_ipc_handle_bytes() bytes, host memory) for the other process to pass to
+ * cp_ipc_open_handle, which returns a device pointer to the peer's memory,
+ * valid in this process until cp_ipc_close_handle. cp_copy_async enqueues one
+ * copy of `bytes` between device pointers, a peer's included (copy engine,
+ * over NVLink between GPUs); it does not wait for the peer, so the caller
+ * orders it against the peer's writes and reads (host barrier plus events).
+ * Errors: CP_ERR_INVALID_ARG (null pointer, zero-byte allocation), CP_ERR_CUDA.
+ */
+CP_API int cp_ring_buffer_alloc(size_t bytes, void** out);
+CP_API int cp_ring_buffer_free(void* p);
+CP_API int cp_ipc_handle_bytes(void);
+CP_API int cp_ipc_get_handle(const void* base, void* handle_out);
+CP_API int cp_ipc_open_handle(const void* handle, void** base_out);
+CP_API int cp_ipc_close_handle(void* base);
+CP_API int cp_copy_async(void* dst, const void* src, size_t bytes, cp_stream_t stream);
+
+/*
  * Backward pass: dQ, dK, dV from the forward's saved O and lse. The pages train
  * long-context models but print no backward; it is the chain rule of the
  * forward's softmax attention (page "Tensor并行与算子拆分", section

@@ -1,0 +1,151 @@
+"""GPU checks of the ring's rank-local path against the oracle.
+
+* ``cp_attn_fwd_ring_step``: every (rank, step) partial, computed from rank-local
+  buffers, against the oracle's ring partial of that rank and step;
+* the whole ring (``ring.RingRank``): N ranks emulated as host threads of one
+  process on one GPU, each with its own compute and copy streams, pulling the
+  next rank's slots by copy engine and meeting at a host barrier every step; each
+  rank's rows against the oracle's full attention, and against the fused
+  single-launch forward on the 4k zigzag workload;
+* the IPC plumbing that can run in one process (handles, device views).
+The rank processes of a real multi-GPU ring need one GPU each; their protocol is
+checked on CPU with gloo processes (tests/test_ring_host.py).
+"""
+import numpy as np
+import pytest
+import torch
+
+import context_long_sequence_cp_b200 as cp
+from context_long_sequence_cp_b200 import ring as R
+from oracle import attention as A
+from oracle import layouts as L
+from tests import gpu_util as G
+from workloads import WORKLOADS, make_qkv, make_small
+
+pytestmark = pytest.mark.gpu
+
+
+def _rank_inputs(x, N, layout):
+    """natural [B, S, H, D] -> per-rank contiguous [B, S/N, H, D] tensors on the GPU."""
+    y = G.to_layout(x, N, layout).cuda()
+    return [y[r].contiguous() for r in range(N)]
+
+
+@pytest.mark.parametrize("B,H,S,D,N,layout,causal", [
+    (1, 2, 256, 64, 4, "contiguous", False),
+    (1, 2, 1024, 128, 4, "zigzag", True),
+    (2, 2, 1536, 64, 3, "contiguous", True),
+    (1, 3, 1920, 128, 5, "zigzag", True),      # 384 local tokens: a ragged query-tile pair
+])
+def test_ring_step_matches_oracle_partials(B, H, S, D, N, layout, causal):
+    q, k, v = make_small(B, H, S, D, 60 + N)
+    plan = cp.Plan(B, H, S, D, N, causal, layout)
+    qs, ks, vs = (_rank_inputs(x, N, layout) for x in (q, k, v))
+    f = lambda t: t.float().numpy()
+    parts = A.ring_partials(f(q), f(k), f(v), L.rank_major_map(B, S, N, layout), N, causal=causal)
+    T = S // N
+    for r in range(N):
+        for t in range(N):
+            rk = (r + t) % N
+            op, lp = cp.attn_fwd_ring_step(plan, r, t, qs[r], ks[rk], vs[rk])
+            assert cp.check(plan) == 0
+            op = op.double().cpu().numpy().reshape(B, T, H, D)
+            lp = lp.double().cpu().numpy().reshape(B, T, H)
+            o_ref = parts[r][t][0]
+            l_ref = parts[r][t][1].transpose(0, 2, 1)
+            fin = np.isfinite(l_ref)
+            assert np.array_equal(np.isfinite(lp), fin), (r, t)
+            assert np.all(op[~fin] == 0)
+            d = np.abs(op - o_ref)
+            assert d.max() <= G.TOL_O_MAX and d.mean() <= G.TOL_O_MEAN, (r, t, d.max())
+            if fin.any():
+                assert np.abs(lp[fin] - l_ref[fin]).max() <= G.TOL_LSE
+
+
+def _run_ring(plan, qs, ks, vs, reps=1):
+    ranks = R.thread_ring(plan)
+    try:
+        for _ in range(reps):
+            out = R.run_threads(ranks, list(zip(qs, ks, vs)))
+        torch.cuda.synchronize()
+        assert cp.check(plan) == 0
+        return [(o.clone(), l.clone()) for o, l in out]
+    finally:
+        for rr in ranks:
+            rr.close()
+
+
+@pytest.mark.parametrize("B,H,S,D,N,layout,causal", [
+    (1, 2, 256, 64, 4, "contiguous", False),
+    (1, 2, 2048, 128, 4, "zigzag", True),
+    (2, 2, 1536, 64, 3, "contiguous", True),
+    (1, 2, 1024, 128, 2, "zigzag", True),
+    (1, 2, 512, 128, 1, "contiguous", True),
+])
+def test_ring_threads_match_oracle(B, H, S, D, N, layout, causal):
+    q, k, v = make_small(B, H, S, D, 70 + N)
+    plan = cp.Plan(B, H, S, D, N, causal, layout)
+    qs, ks, vs = (_rank_inputs(x, N, layout) for x in (q, k, v))
+    out = _run_ring(plan, qs, ks, vs, reps=2)       # the second call reuses the slots
+    f = lambda t: t.float().numpy()
+    o_ref, lse_ref = A.attention(f(q), f(k), f(v), causal=causal)       # [B, S, H, D], [B, H, S]
+    pos = L.chunk_positions(S, N, layout)
+    T = S // N
+    for r in range(N):
+        o, lse = out[r]
+        o = o.double().cpu().numpy()                                     # [B, T, H, D]
+        lse = lse.double().cpu().numpy().reshape(B, T, H)
+        d = np.abs(o - o_ref[:, pos[r]])
+        assert d.max() <= G.TOL_O_MAX and d.mean() <= G.TOL_O_MEAN, (r, d.max())
+        assert np.abs(lse - lse_ref[:, :, pos[r]].transpose(0, 2, 1)).max() <= G.TOL_LSE
+
+
+def test_ring_threads_match_fused_zigzag_4k():
+    w = WORKLOADS["zigzag_4k"]
+    q, k, v = make_qkv(w)
+    plan = cp.Plan(w.B, w.H, w.S, w.D, w.N, w.causal, w.layout)
+    qd, kd, vd = (G.to_layout(x, w.N, w.layout).cuda() for x in (q, k, v))
+    o_f, lse_f = cp.attn_fwd(plan, qd, kd, vd)
+    out = _run_ring(plan, [qd[r].contiguous() for r in range(w.N)], [kd[r].contiguous() for r in range(w.N)],
+                    [vd[r].contiguous() for r in range(w.N)])
+    T = w.S // w.N
+    pos = L.chunk_positions(w.S, w.N, w.layout)
+    for r in range(w.N):
+        o, lse = out[r]
+        d = (o.float() - o_f[r].float()).abs()
+        assert d.max().item() <= G.TOL_O_MAX and d.mean().item() <= G.TOL_O_MEAN
+        l_f = lse_f[:, :, torch.from_numpy(pos[r]).cuda()].permute(0, 2, 1)      # [B, T, H]
+        assert (lse.reshape(w.B, T, w.H) - l_f).abs().max().item() <= G.TOL_LSE
+    # sampled rows of rank 0 and the last rank against the oracle too
+    rows = np.array([[0, h, int(p)] for h in (0, w.H - 1) for p in (pos[0, 5], pos[0, -1], pos[-1, 7], pos[-1, -3])])
+    o_ref, l_ref = G.oracle_rows(q, k, v, rows, w.causal)
+    o_nat = G.from_layout(torch.stack([o for o, _ in out]), w.N, w.layout)
+    ix = [torch.from_numpy(rows[:, j]).cuda() for j in (0, 2, 1)]
+    got = o_nat[ix[0], ix[1], ix[2]].double().cpu().numpy()
+    assert np.abs(got - o_ref).max() <= G.TOL_O_MAX
+
+
+def test_ring_buffers_and_ipc_handle():
+    buf = cp.DeviceBuffer(1 << 20)
+    try:
+        h = buf.ipc_handle()
+        assert len(h) == 64 and any(h)
+        t = buf.view((512, 1024), torch.bfloat16, device="cuda")
+        t.copy_(torch.arange(512 * 1024, device="cuda").reshape(512, 1024).to(torch.bfloat16))
+        dst = torch.empty(512, 1024, dtype=torch.bfloat16, device="cuda")
+        cp.copy_async(dst.data_ptr(), buf.ptr, 1 << 20)
+        torch.cuda.synchronize()
+        assert torch.equal(dst.view(torch.int16), t.view(torch.int16))
+    finally:
+        buf.close()
+
+
+def test_ring_step_rejects_bad_arguments():
+    plan = cp.Plan(1, 2, 1024, 64, 4, True, "zigzag")
+    x = torch.zeros(1, 256, 2, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(cp.CpAttnError) as e:
+        cp.attn_fwd_ring_step(plan, 4, 0, x, x, x)
+    assert e.value.status == -1
+    with pytest.raises(cp.CpAttnError) as e:
+        cp.attn_fwd_ring_step(plan, 0, 0, x.view(-1)[1:], x, x)      # 2 bytes past a 16-byte boundary
+    assert e.value.status == -3
