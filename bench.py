@@ -384,6 +384,67 @@ def main():
     if cp.check(plan) != 0:
         raise RuntimeError("component runs failed")
 
+    # --- one rank of the multi-GPU ring on its own GPU: rank 0 of N, the other
+    # ranks' own K/V blocks read from the layout tensors, standing in for their
+    # slot buffers (on N GPUs: their memory over NVLink). The ring driver runs as
+    # on N GPUs: fill of the own slot, one host barrier, ONE cooperative launch
+    # whose copy warps fetch the other blocks in ring order while its units
+    # compute step-major, then the merge. Compared with the same launch on
+    # resident blocks (no fetch), with one launch per ring step, and with 1/N of
+    # the fused launch (the rank's share of the one-GPU forward). L2 is flushed
+    # before every timed call.
+    from context_long_sequence_cp_b200 import ring as R
+
+    class _OneRank(R.RingRank):
+        def pull_sources(self, c):
+            return [kz[j].data_ptr() for j in range(N)], [vz[j].data_ptr() for j in range(N)]
+
+    blk = kz[0].numel() * 2
+    q0 = qz[0]
+    ro = torch.empty(plan.rows // N, D, dtype=torch.bfloat16, device=dev)
+    rl = torch.empty(plan.rows // N, dtype=torch.float32, device=dev)
+    l2_flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def time_flushed(fn, reps=5):
+        out = []
+        for i in range(reps + 1):
+            l2_flush.zero_()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            fn()
+            a1.record(stream)
+            torch.cuda.synchronize(dev)
+            if i > 0:
+                out.append(a0.elapsed_time(a1))
+        return statistics.median(out)
+
+    rr = _OneRank(plan, 0, barrier=lambda: None)
+    rr.connect([0] * N)
+    for _ in range(2):                    # both slot sets
+        r_o, _ = rr.forward(q0, kz[0], vz[0], stream)
+        torch.cuda.synchronize(dev)
+        ring_err = (r_o.float() - oz[0].float()).abs().max().item()
+        if cp.check(plan) != 0 or not ring_err <= 2e-2:
+            raise RuntimeError(f"ring rank 0 disagrees with the fused forward: {ring_err}")
+    ring_ms = time_flushed(lambda: rr.forward(q0, kz[0], vz[0], stream))
+    op_r, lp_r = rr.o_parts, rr.lse_parts
+
+    def launch_only():
+        cp.attn_fwd_ring(plan, 0, q0, kz, vz, o_parts=op_r, lse_parts=lp_r, stream=stream)
+        cp.merge_partials(op_r, lp_r, o_out=ro, lse_out=rl)
+
+    def step_launches():
+        for t in range(N):
+            cp.attn_fwd_ring_step(plan, 0, t, q0, kz[t], vz[t], op_r[t], lp_r[t], stream)
+        cp.merge_partials(op_r, lp_r, o_out=ro, lse_out=rl)
+
+    ring_launch_ms = time_flushed(launch_only)
+    ring_steps_ms = time_flushed(step_launches)
+    if cp.check(plan) != 0:
+        raise RuntimeError("ring runs failed")
+    rr.close()
+    del l2_flush
+
     # --- end to end through the public API from pinned host buffers. Every step
     # uploads its own Q/K/V from pinned memory and reads back its own O and lse;
     # as a user of the API would, the steps are pipelined: uploads run on one copy
@@ -490,6 +551,16 @@ def main():
             "partials_ms": part_ms, "merge_ms": merge_ms, "merge_gbs": merge_gbs,
             "merge_frac_hbm": merge_gbs / float(peaks["hbm_gbs"]),
             "unfused_tflops": w.flops / ((part_ms + merge_ms) * 1e-3) / 1e12,
+            "ring_rank_ms": ring_ms, "ring_rank_tflops": w.flops / N / (ring_ms * 1e-3) / 1e12,
+            "ring_rank_launch_only_ms": ring_launch_ms, "ring_rank_step_launches_ms": ring_steps_ms,
+            "ring_rank_fused_share_ms": att / N,
+            "ring_overhead_vs_fused_share": ring_ms / (att / N) - 1.0,
+            "ring_fetch_cost": ring_ms / ring_launch_ms - 1.0,
+            "ring_fetch_bytes": (N - 1) * 2 * blk,
+            "ring_note": f"rank 0 of {N} on one GPU: fill + one cooperative launch whose copy warps fetch the "
+                         f"other {N - 1} K/V blocks ({(N - 1) * 2 * blk >> 20} MiB; here from local HBM, on N "
+                         "GPUs over NVLink) while its units compute, + merge; launch_only = blocks resident; "
+                         "step_launches = one launch per ring step; fused_share = the fused launch / N",
         },
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e_ms, "pipelined": "uploads, step and read-backs of consecutive steps overlap "

@@ -49,6 +49,7 @@ SIGNATURES = {
     "cp_attn_fwd_ulysses_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P]),
     "cp_attn_fwd_ring_step": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _P]),
     "cp_attn_ring_prepare": (_I, [_P, _I]),
+    "cp_attn_fwd_ring": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "cp_attn_ring_schedule": (_I64, [_P, _I, _I, _P, _P]),
     "cp_ring_buffer_alloc": (_I, [_SZ, ctypes.POINTER(_P)]),
     "cp_ring_buffer_free": (_I, [_P]),
@@ -168,7 +169,8 @@ class Plan:
 
     def ring_schedule(self, rank: int, step: int):
         """Schedule of one rank's ring step: (items as rows of (row block, head,
-        query-tile pair, key tiles, CTA) in run order, per-CTA modelled loads)."""
+        query-tile pair, key tiles, CTA) in run order, per-CTA modelled loads);
+        step -1: the units of the one-launch ring forward (pair | step << 16)."""
         n = int(lib().cp_attn_ring_schedule(self._h, int(rank), int(step), None, None))
         if n < 0:
             raise CpAttnError("cp_attn_ring_schedule", n)
@@ -230,6 +232,34 @@ def attn_fwd_ring_step(plan: Plan, rank: int, step: int, q, k, v, o_part=None, l
            lib().cp_attn_fwd_ring_step(plan.handle, int(rank), int(step), _ptr(q), _ptr(k), _ptr(v), _ptr(o_part),
                                        _ptr(lse_part), _stream(stream)))
     return o_part, lse_part
+
+
+def attn_fwd_ring(plan: Plan, rank: int, q, k_all, v_all, pull_k=None, pull_v=None, arrived=None,
+                  o_parts=None, lse_parts=None, stream=None):
+    """``cp_attn_fwd_ring``: all N step partials of rank ``rank`` in one launch.
+
+    k_all, v_all: [N, B, S/N, H, D] tensors or device addresses (slot j = rank
+    j's block; slot ``rank`` filled). pull_k, pull_v: N device addresses of the
+    ranks' own blocks to fetch from (None: every slot already filled). arrived:
+    int32 [N] device tensor (needed when pulling). Returns (o_parts fp32
+    [N, rows, D], lse_parts fp32 [N, rows]), rows = B*(S/N)*H."""
+    rows = plan.B * (plan.S // plan.N) * plan.H
+    if o_parts is None:
+        o_parts = torch.empty(plan.N, rows, plan.D, dtype=torch.float32, device=q.device)
+    if lse_parts is None:
+        lse_parts = torch.empty(plan.N, rows, dtype=torch.float32, device=q.device)
+    pk = None if pull_k is None else (ctypes.c_void_p * len(pull_k))(*[int(x) for x in pull_k])
+    pv = None if pull_v is None else (ctypes.c_void_p * len(pull_v))(*[int(x) for x in pull_v])
+    as_ptr = lambda a: None if a is None else ctypes.cast(a, ctypes.c_void_p)
+    _check("cp_attn_fwd_ring",
+           lib().cp_attn_fwd_ring(plan.handle, int(rank), _ptr(q), _vp_of(k_all), _vp_of(v_all), as_ptr(pk),
+                                  as_ptr(pv), None if arrived is None else _vp_of(arrived), _ptr(o_parts),
+                                  _ptr(lse_parts), _stream(stream)))
+    return o_parts, lse_parts
+
+
+def _vp_of(x):
+    return ctypes.c_void_p(int(x) if isinstance(x, int) else x.data_ptr())
 
 
 def copy_async(dst_ptr: int, src_ptr: int, nbytes: int, stream=None):

@@ -75,6 +75,14 @@ struct cp_attn_plan_s {
     std::vector<int64_t> cta_load;    // [NR][sms]
     WorkItem* d_items = nullptr;
     int* d_cta_begin = nullptr;
+    // The rank's whole forward as one launch: every (step, item) unit, step-major
+    // and longest first within a step, assigned to CTAs in that order.
+    std::vector<WorkItem> units;
+    std::vector<int> unit_cta_begin;
+    std::vector<int64_t> unit_cta_load;
+    int unit_n_cta = 0;
+    WorkItem* d_units = nullptr;
+    int* d_unit_cta_begin = nullptr;
   };
   int sms = kDefaultSmCountPlan;
   std::vector<RingRank> ring;
@@ -83,6 +91,7 @@ struct cp_attn_plan_s {
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per in-kernel wait
+constexpr int64_t kPullChunkBytes = 32768;          // fused-pull copy unit
 constexpr int kDefaultSmCount = kDefaultSmCountPlan;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -303,22 +312,58 @@ void build_ring_rank(cp_attn_plan_s* p, int r) {
     std::copy(load.begin(), load.end(), rr.cta_load.begin() + static_cast<size_t>(t) * p->sms);
     rr.items.insert(rr.items.end(), items.begin(), items.end());
   }
+  // One launch over all steps: the units of step t follow those of step t - 1,
+  // so that the CTAs reach a block in about the order the blocks arrive.
+  std::vector<WorkItem> units;
+  std::vector<int64_t> cost;
+  units.reserve(rr.items.size());
+  cost.reserve(rr.items.size());
+  for (int t = 0; t < g.NR; ++t)
+    for (int i = 0; i < rr.nper; ++i) {
+      WorkItem w = rr.items[static_cast<size_t>(t) * rr.nper + i];
+      cost.push_back(2 * static_cast<int64_t>(w.cost) + kItemOverheadHalfTiles);
+      w.qp = pack_unit_qp(w.qp, t);
+      units.push_back(w);
+    }
+  // rr.items is grouped by CTA within each step; restore the longest-first order
+  std::vector<size_t> order(units.size());
+  for (size_t i = 0; i < order.size(); ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(), [&](size_t a, size_t b) {
+    const int ta = item_step(units[a]), tb = item_step(units[b]);
+    if (ta != tb) return ta < tb;
+    return cost[a] > cost[b];
+  });
+  rr.units.clear();
+  std::vector<int64_t> ucost;
+  for (size_t i : order) {
+    rr.units.push_back(units[i]);
+    ucost.push_back(cost[i]);
+  }
+  rr.unit_n_cta = assign_greedy(rr.units, ucost, p->sms, rr.unit_cta_begin, rr.unit_cta_load);
   rr.built = true;
 }
 
 void free_ring(cp_attn_plan_s::RingRank& rr) {
-  if (rr.d_items != nullptr) cudaFree(rr.d_items);
-  if (rr.d_cta_begin != nullptr) cudaFree(rr.d_cta_begin);
+  for (void* ptr : {static_cast<void*>(rr.d_items), static_cast<void*>(rr.d_cta_begin),
+                    static_cast<void*>(rr.d_units), static_cast<void*>(rr.d_unit_cta_begin)})
+    if (ptr != nullptr) cudaFree(ptr);
   rr.d_items = nullptr;
   rr.d_cta_begin = nullptr;
+  rr.d_units = nullptr;
+  rr.d_unit_cta_begin = nullptr;
 }
 
 int upload_ring_rank(cp_attn_plan_s::RingRank& rr) {
   if (rr.d_items != nullptr) return CP_OK;
   const size_t ib = rr.items.size() * sizeof(WorkItem), cb = rr.cta_begin.size() * sizeof(int);
+  const size_t ub = rr.units.size() * sizeof(WorkItem), ucb = rr.unit_cta_begin.size() * sizeof(int);
   const bool ok = cudaMalloc(&rr.d_items, ib) == cudaSuccess && cudaMalloc(&rr.d_cta_begin, cb) == cudaSuccess &&
+                  cudaMalloc(&rr.d_units, ub) == cudaSuccess && cudaMalloc(&rr.d_unit_cta_begin, ucb) == cudaSuccess &&
                   cudaMemcpy(rr.d_items, rr.items.data(), ib, cudaMemcpyHostToDevice) == cudaSuccess &&
-                  cudaMemcpy(rr.d_cta_begin, rr.cta_begin.data(), cb, cudaMemcpyHostToDevice) == cudaSuccess;
+                  cudaMemcpy(rr.d_cta_begin, rr.cta_begin.data(), cb, cudaMemcpyHostToDevice) == cudaSuccess &&
+                  cudaMemcpy(rr.d_units, rr.units.data(), ub, cudaMemcpyHostToDevice) == cudaSuccess &&
+                  cudaMemcpy(rr.d_unit_cta_begin, rr.unit_cta_begin.data(), ucb, cudaMemcpyHostToDevice) ==
+                      cudaSuccess;
   if (!ok) {
     free_ring(rr);
     return CP_ERR_CUDA;
@@ -699,9 +744,25 @@ int cp_attn_ring_prepare(cp_attn_plan_t plan, int rank) {
 int64_t cp_attn_ring_schedule(cp_attn_plan_t plan, int rank, int step, int32_t* items, int64_t* cta_loads) {
   if (plan == nullptr) return CP_ERR_INVALID_ARG;
   if (plan->layout == CP_LAYOUT_ULYSSES) return CP_ERR_UNSUPPORTED;
-  if (rank < 0 || rank >= plan->N || step < 0 || step >= plan->N) return CP_ERR_INVALID_ARG;
+  if (rank < 0 || rank >= plan->N || step < -1 || step >= plan->N) return CP_ERR_INVALID_ARG;
   cp_attn_plan_s::RingRank& rr = plan->ring[rank];
   if (!rr.built) build_ring_rank(plan, rank);
+  if (step == -1) {   // the one-launch schedule of cp_attn_fwd_ring
+    const int n_cta = rr.unit_n_cta;
+    if (items != nullptr)
+      for (int c = 0; c < n_cta; ++c)
+        for (int i = rr.unit_cta_begin[c]; i < rr.unit_cta_begin[c + 1]; ++i) {
+          int32_t* o = items + static_cast<size_t>(i) * 5;
+          o[0] = rr.units[i].rb;
+          o[1] = rr.units[i].h;
+          o[2] = rr.units[i].qp;
+          o[3] = rr.units[i].cost;
+          o[4] = c;
+        }
+    if (cta_loads != nullptr)
+      for (int c = 0; c < n_cta; ++c) cta_loads[c] = rr.unit_cta_load[c];
+    return static_cast<int64_t>(rr.units.size());
+  }
   const int stride = plan->sms + 1;
   const int* cb = rr.cta_begin.data() + static_cast<size_t>(step) * stride;
   const WorkItem* it = rr.items.data() + static_cast<size_t>(step) * rr.nper;
@@ -758,6 +819,76 @@ int cp_attn_fwd_ring_step(cp_attn_plan_t plan, int rank, int step, const void* q
   P.status = plan->d_status;
   P.wait_limit_ns = kWaitLimitNs;
   return launch_attn_fwd(L, plan->D, true, static_cast<cudaStream_t>(stream)) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+int cp_attn_fwd_ring(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all,
+                     const void* const* pull_k, const void* const* pull_v, int* arrived, float* o_parts,
+                     float* lse_parts, cp_stream_t stream) {
+  if (plan == nullptr || q == nullptr || k_all == nullptr || v_all == nullptr || o_parts == nullptr ||
+      lse_parts == nullptr)
+    return CP_ERR_INVALID_ARG;
+  if (plan->layout == CP_LAYOUT_ULYSSES) return CP_ERR_UNSUPPORTED;
+  if (rank < 0 || rank >= plan->N) return CP_ERR_INVALID_ARG;
+  if ((pull_k == nullptr) != (pull_v == nullptr)) return CP_ERR_INVALID_ARG;
+  const bool pull = pull_k != nullptr && plan->N > 1;
+  if (pull && arrived == nullptr) return CP_ERR_INVALID_ARG;
+  if (pull && plan->N > kMaxPullRanks) return CP_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_all) || !aligned16(v_all) || !aligned16(o_parts) || !aligned16(lse_parts) ||
+      (reinterpret_cast<uintptr_t>(arrived) & 3u))
+    return CP_ERR_ALIGNMENT;
+  const Geometry& g = plan->g;
+  FwdLaunch L;
+  std::memset(&L, 0, sizeof(L));
+  FwdParams& P = L.params;
+  const int64_t block_bytes = static_cast<int64_t>(g.B) * g.T * g.Hh * plan->D * 2;
+  if (pull) {
+    for (int j = 0; j < plan->N; ++j) {
+      if (j == rank) continue;
+      if (pull_k[j] == nullptr || pull_v[j] == nullptr) return CP_ERR_INVALID_ARG;
+      if (!aligned16(pull_k[j]) || !aligned16(pull_v[j])) return CP_ERR_ALIGNMENT;
+      P.pull_src[2 * j] = reinterpret_cast<uint64_t>(pull_k[j]);
+      P.pull_src[2 * j + 1] = reinterpret_cast<uint64_t>(pull_v[j]);
+    }
+    const int64_t chunk = block_bytes < kPullChunkBytes ? block_bytes : kPullChunkBytes;
+    const int64_t per_half = (block_bytes + chunk - 1) / chunk;
+    if (2 * per_half > (int64_t(1) << 30)) return CP_ERR_UNSUPPORTED;
+    P.pull_k_all = static_cast<char*>(k_all);
+    P.pull_v_all = static_cast<char*>(v_all);
+    P.pull_block_bytes = block_bytes;
+    P.pull_chunk_bytes = static_cast<int>(chunk);
+    P.pull_chunks = static_cast<int>(2 * per_half);
+  }
+  int rc = ensure_device(plan);
+  if (rc != CP_OK) return rc;
+  if ((rc = cp_attn_ring_prepare(plan, rank)) != CP_OK) return rc;
+  const cp_attn_plan_s::RingRank& rr = plan->ring[rank];
+  if ((rc = encode_view(&L.tm_q, q, g, plan->D, g.B)) != CP_OK) return rc;
+  if ((rc = encode_view(&L.tm_k, k_all, g, plan->D)) != CP_OK) return rc;
+  if ((rc = encode_view(&L.tm_v, v_all, g, plan->D)) != CP_OK) return rc;
+  P.g = g;
+  P.t_begin = 0;
+  P.t_end = g.NR;
+  P.scale_log2 = plan->scale * 1.4426950408889634f;
+  P.items = rr.d_units;
+  P.n_items = static_cast<int>(rr.units.size());
+  P.cta_begin = rr.d_unit_cta_begin;
+  P.n_cta = rr.unit_n_cta;
+  P.step_off = plan->d_step_off;
+  P.entries = plan->d_entries;
+  P.npairs = plan->npairs;
+  P.o_part = o_parts;
+  P.lse_part = lse_parts;
+  P.q_rb0 = rank * g.B;
+  P.kv_local = 0;
+  P.unit_steps = 1;
+  P.part_rows = static_cast<int64_t>(g.B) * g.T * g.Hh;
+  P.arrived = arrived;
+  P.arrive_target = pull ? P.pull_chunks : 1;
+  P.status = plan->d_status;
+  P.wait_limit_ns = kWaitLimitNs;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (pull && cudaMemsetAsync(arrived, 0, sizeof(int) * plan->N, st) != cudaSuccess) return CP_ERR_CUDA;
+  return launch_attn_fwd(L, plan->D, true, st) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
 int cp_merge_partials(int num_parts, int64_t rows, int D, const float* o_parts, const float* lse_parts,

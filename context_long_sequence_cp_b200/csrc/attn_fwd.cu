@@ -173,6 +173,21 @@ __device__ __forceinline__ void rescale_p_half(uint32_t tS, float beta) {
 
 }  // namespace
 
+// Walk of an item: its precomputed key tiles over ring steps [t_begin, t_end),
+// or over its own step for the units of a ring launch.
+template <bool PARTIAL>
+__device__ __forceinline__ void item_walk(const FwdParams& p, const WorkItem& w, int rq, int& e_begin, int& e_end) {
+  const int qp = PARTIAL ? item_qp(w) : w.qp;
+  const int* off = p.step_off + (rq * p.npairs + qp) * (p.g.NR + 1);
+  int t0 = p.t_begin, t1 = p.t_end;
+  if (PARTIAL && p.unit_steps) {
+    t0 = item_step(w);
+    t1 = t0 + 1;
+  }
+  e_begin = __ldg(off + t0);
+  e_end = __ldg(off + t1);
+}
+
 template <int D, bool PARTIAL>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -220,7 +235,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int it_end = __ldg(p.cta_begin + blockIdx.x + 1);   // this CTA's items end here
 
   // Every role walks the same precomputed key list of each work item.
-  const int nstep_off = g.NR + 1;
 
   if (warp == 9) {
     // ------------------------------------------------------------ TMA producer
@@ -235,9 +249,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const WorkItem w = p.items[it];
         const int rq = w.rb / g.B;
         const int bv = w.rb - rq * g.B;
-        const int q0 = w.qp * kPair;
-        const int* off = p.step_off + (rq * p.npairs + w.qp) * nstep_off;
-        const int e_begin = __ldg(off + p.t_begin), e_end = __ldg(off + p.t_end);
+        const int q0 = (PARTIAL ? item_qp(w) : w.qp) * kPair;
+        int e_begin, e_end;
+        item_walk<PARTIAL>(p, w, rq, e_begin, e_end);
+        if (PARTIAL && p.arrived != nullptr && e_begin < e_end) {
+          // another rank's block: wait until all of it has arrived
+          const int rk = entry_rank(__ldg(p.entries + e_begin));
+          if (rk != rq) ok = count_wait(p.arrived + rk, p.arrive_target, ctl);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+        }
         if (q_iter > 0) ok = mbar_wait(smem_addr(&sm.q_empty), (q_iter - 1) & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
@@ -290,8 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = __ldg(p.cta_begin + blockIdx.x); it < it_end && ok; ++it) {
         const WorkItem w = p.items[it];
         const int rq = w.rb / g.B;
-        const int* off = p.step_off + (rq * p.npairs + w.qp) * nstep_off;
-        const int e_begin = __ldg(off + p.t_begin), e_end = __ldg(off + p.t_end);
+        int e_begin, e_end;
+        item_walk<PARTIAL>(p, w, rq, e_begin, e_end);
         // The last PV of each query tile signals o_done: find where they are.
         int last0 = -1, last1 = -1;
         for (int e = e_begin; e < e_end; ++e) {
@@ -426,12 +447,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         const WorkItem w = p.items[it];
         const int rq = w.rb / g.B;
-        const int tl = w.qp * kPair + wg * kTile + row;
+        const int tl = (PARTIAL ? item_qp(w) : w.qp) * kPair + wg * kTile + row;
         valid = tl < g.T;
         gq = global_pos(g, rq, valid ? tl : g.T - 1);
-        const int* off = p.step_off + (rq * p.npairs + w.qp) * nstep_off;
-        e_begin = __ldg(off + p.t_begin);
-        e_end = __ldg(off + p.t_end);
+        item_walk<PARTIAL>(p, w, rq, e_begin, e_end);
       }
       float m_run = -INFINITY, l_run = 0.f;
       int ntile = 0;
@@ -521,8 +540,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // across the key loop in registers the scores need.
       const WorkItem w = ld_item_volatile(p.items + it);
       const int bv = w.rb % g.B;
-      const int tl = w.qp * kPair + wg * kTile + row;
-      const int64_t row_id = (static_cast<int64_t>(w.rb - p.q_rb0) * g.T + tl) * g.Hh + w.h;
+      const int tl = (PARTIAL ? item_qp(w) : w.qp) * kPair + wg * kTile + row;
+      const int64_t row_id = (static_cast<int64_t>(w.rb - p.q_rb0) * g.T + tl) * g.Hh + w.h +
+                             (PARTIAL && p.unit_steps ? item_step(w) * p.part_rows : 0);
       if (ntile > 0) {
         ok = mbar_wait(smem_addr(&sm.o_done[wg]), od_cnt & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
@@ -585,6 +605,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  if constexpr (PARTIAL) {
+    if (warp >= 10 && p.pull_chunks > 0) {
+      // ---------------------------------------------------------- fused pull
+      // Copy warps: chunk c of the (NR - 1) * pull_chunks chunks goes to copy
+      // warp c mod (2 * grid), so every warp walks the blocks in ring order and
+      // each block completes at about the same time on all of them.
+      const int cw = static_cast<int>(blockIdx.x) * 2 + (warp - 10);
+      const int ncw = static_cast<int>(gridDim.x) * 2;
+      const int rank = p.q_rb0 / g.B;
+      const int per_half = p.pull_chunks / 2;
+      const int64_t half = p.pull_block_bytes;
+      const int64_t total = static_cast<int64_t>(g.NR - 1) * p.pull_chunks;
+      for (int64_t c = cw; c < total; c += ncw) {
+        if (abort_raised(ctl.wb)) break;
+        const int jj = static_cast<int>(c / p.pull_chunks);
+        const int ci = static_cast<int>(c - static_cast<int64_t>(jj) * p.pull_chunks);
+        int j = rank + 1 + jj;
+        if (j >= g.NR) j -= g.NR;
+        const int is_v = ci >= per_half;
+        const int64_t off = static_cast<int64_t>(ci - is_v * per_half) * p.pull_chunk_bytes;
+        const int64_t n = half - off < p.pull_chunk_bytes ? half - off : p.pull_chunk_bytes;
+        const char* src = reinterpret_cast<const char*>(p.pull_src[2 * j + is_v]) + off;
+        char* dst = (is_v ? p.pull_v_all : p.pull_k_all) + static_cast<int64_t>(j) * half + off;
+        constexpr int kU = 8;   // 16-byte vectors in flight per lane
+        for (int64_t i = static_cast<int64_t>(lane) * 16; i < n; i += 32 * 16 * kU) {
+          uint4 r[kU];
+#pragma unroll
+          for (int u = 0; u < kU; ++u)
+            if (i + u * 512 < n) r[u] = ld_stream_v4(src + i + u * 512);
+#pragma unroll
+          for (int u = 0; u < kU; ++u)
+            if (i + u * 512 < n) st_v4(dst + i + u * 512, r[u]);
+        }
+        chunk_stores_fence();
+        __syncwarp();
+        if (lane == 0) red_release_add(p.arrived + j, 1);
+      }
+    }
+  }
+
   tc_fence_before();
   __syncthreads();
   if (warp == 8) {
@@ -606,8 +666,19 @@ cudaError_t launch_impl(const FwdLaunch& L, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const int grid = L.params.n_cta;   // the schedule's CTA count (normally the SM count)
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, kThreads, smem, stream>>>(L.tm_q, L.tm_k, L.tm_v, L.params);
-  return cudaGetLastError();
+  // A fused-pull launch is cooperative: units wait for chunks that copy warps of
+  // other CTAs bring in, so all CTAs must be resident together (one per SM).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (PARTIAL && L.params.pull_chunks > 0) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, L.tm_q, L.tm_k, L.tm_v, L.params);
 }
 
 }  // namespace

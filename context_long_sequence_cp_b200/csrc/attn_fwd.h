@@ -11,6 +11,8 @@
 
 namespace cpattn {
 
+constexpr int kMaxPullRanks = 64;   // ranks a fused-pull ring launch can fetch from
+
 struct FwdParams {
   Geometry g;
   int t_begin, t_end;          // ring steps visited: [t_begin, t_end)
@@ -35,6 +37,26 @@ struct FwdParams {
   // v maps hold the key rank's B row blocks only.
   int q_rb0;
   int kv_local;
+  // Ring launches (partial mode): every item is a (ring step, item) unit whose
+  // partial goes to part item_step(w), part_rows rows per part; before reading
+  // the key/value block of another rank k the producer waits until arrived[k]
+  // >= arrive_target (arrived null: no wait).
+  int unit_steps;
+  int64_t part_rows;
+  int* arrived;
+  int arrive_target;
+  // Fused pull (ring launches): warps 10 and 11 of every CTA copy the blocks of
+  // the other ranks, in ring order from the query rank, from pull_src[2k] (K)
+  // and pull_src[2k + 1] (V) into slot k of pull_k_all / pull_v_all, in chunks of
+  // pull_chunk_bytes, adding 1 to arrived[k] per finished chunk; pull_chunks
+  // chunks per block, K and V together (0: no pull). The launch is cooperative,
+  // so every CTA whose chunks a unit waits for is resident.
+  uint64_t pull_src[2 * kMaxPullRanks];
+  char* pull_k_all;
+  char* pull_v_all;
+  int64_t pull_block_bytes;
+  int pull_chunk_bytes;
+  int pull_chunks;
   int* status;                 // device status word (0 = ok)
   uint64_t wait_limit_ns;      // budget of one in-kernel wait
 };

@@ -91,6 +91,12 @@ struct WorkItem {
   int cost;  // executed key tiles (both query tiles), used for ordering
 };
 
+// Ring launches run one rank's (ring step, item) units, the step in the high
+// half of qp; everywhere else the high half is zero.
+CP_HD int item_qp(const WorkItem& w) { return w.qp & 0xffff; }
+CP_HD int item_step(const WorkItem& w) { return static_cast<int>(static_cast<unsigned>(w.qp) >> 16); }
+CP_HD int pack_unit_qp(int qp, int step) { return qp | (step << 16); }
+
 // A precomputed key-tile entry of a work item's walk, packed in 32 bits:
 // bits [0,13) key tile index, [13,25) key rank, [25,27) class of query tile 0,
 // [27,29) class of query tile 1.

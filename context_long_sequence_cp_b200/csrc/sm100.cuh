@@ -117,6 +117,71 @@ static __device__ __noinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parit
   }
 }
 
+// Arrival count of a block, raised by the copy warps of this kernel (release
+// adds after each finished chunk): wait until it reaches `target`, then order the
+// async proxy (TMA loads of the block) after that observation. Same budget and
+// abort flag as the mbarrier waits; false on abort/timeout. Every lane of the
+// calling warp polls the same word.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ bool abort_raised(uint32_t wb) {
+  int ab;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(ab) : "r"(wb + 16));
+  return ab != 0;
+}
+
+static __device__ __noinline__ bool count_wait_slow(const int* count, int target, uint32_t wb) {
+  const uint64_t t0 = globaltimer_ns();
+  uint64_t limit;
+  asm volatile("ld.shared.u64 %0, [%1];" : "=l"(limit) : "r"(wb + 8));
+  for (;;) {
+    if (ld_acquire_gpu(count) >= target) return true;
+    if (abort_raised(wb)) return false;
+    if (globaltimer_ns() - t0 > limit) {
+      asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(wb + 16), "r"(1) : "memory");
+      uint64_t st;
+      asm volatile("ld.shared.u64 %0, [%1];" : "=l"(st) : "r"(wb));
+      atomicCAS(reinterpret_cast<int*>(st), 0, kStatusTimeout);
+      return false;
+    }
+    __nanosleep(256);
+  }
+}
+
+__device__ __forceinline__ bool count_wait(const int* count, int target, WaitCtl ctl) {
+  const bool ok = ld_acquire_gpu(count) >= target || count_wait_slow(count, target, ctl.wb);
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return ok;
+}
+
+// Publish a finished chunk: order this thread's stores before later async-proxy
+// reads (other CTAs' TMA loads) and at GPU scope; after a __syncwarp one lane
+// adds 1 to the block's arrival count with release semantics.
+__device__ __forceinline__ void chunk_stores_fence() {
+  asm volatile("fence.proxy.async.global;\n\tfence.acq_rel.gpu;" ::: "memory");
+}
+__device__ __forceinline__ void red_release_add(int* count, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(count), "r"(v) : "memory");
+}
+
+// 16-byte streaming load (read-only for the kernel's lifetime, no L1 allocation)
+// and store.
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ void st_v4(void* p, const uint4& v) {
+  asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx_elect(uint32_t bar, uint32_t bytes) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"

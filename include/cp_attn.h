@@ -190,8 +190,46 @@ CP_API int cp_attn_fwd_partials(cp_attn_plan_t plan, const void* q, const void* 
 CP_API int cp_attn_fwd_ring_step(cp_attn_plan_t plan, int rank, int step, const void* q, const void* k,
                                  const void* v, float* o_part, float* lse_part, cp_stream_t stream);
 
+/*
+ * One rank's whole ring forward in one launch, fetching the other ranks' blocks
+ * itself. Page "序列与上下文并行", section "上下文并行：注意力本身切分": the rank
+ * computes on the blocks it holds while the next ones arrive. The units (ring
+ * step, pair of query tiles) run step-major on persistent CTAs, starting on the
+ * rank's own block; meanwhile two copy warps of every CTA fetch the blocks of
+ * ranks rank+1, rank+2, ... (mod N), in that order, in 32 KiB chunks, from
+ * pull_k[j] / pull_v[j] into slot j of k_all / v_all, counting finished chunks in
+ * arrived[j]; a unit reads slot j once all of its chunks have arrived. The
+ * launch is cooperative (all CTAs resident), so every wait ends. Behind NVSwitch
+ * pull_k[j] is rank j's own block in its memory, mapped here (cp_ipc_open_handle):
+ * each block crosses NVLink once, by loads of the copy warps, with no copy
+ * engine or stream between the transfer and the math.
+ *   q            : bf16 [B][S/N][H][D], this rank's own chunk, device
+ *   k_all, v_all : bf16 [N][B][S/N][H][D] (written: the pulled slots); slot
+ *                  `rank` holds the rank's own block before the launch, device
+ *   pull_k, pull_v : host arrays of N device pointers, entry j = rank j's own
+ *                  K/V block [B][S/N][H][D] as addressable from this GPU (entry
+ *                  `rank` unused), 16-byte aligned, unchanged until the kernel
+ *                  ends; both NULL: no pull, every slot already holds its block
+ *   arrived      : int32 [N] device workspace (set to 0 on `stream` before the
+ *                  launch when pulling). Without pull sources and with arrived
+ *                  not NULL, a unit waits until arrived[j] >= 1, written by the
+ *                  caller from outside this GPU's SMs (not by a copy that needs
+ *                  them: the persistent kernel holds every SM)
+ *   o_parts      : float32 [N][B*(S/N)*H][D], part t = step t, device (written)
+ *   lse_parts    : float32 [N][B*(S/N)*H], device (written)
+ * Rows as in cp_attn_fwd_ring_step; cp_merge_partials over the N parts gives the
+ * rank's rows of full attention. Errors: as cp_attn_fwd_ring_step;
+ * CP_ERR_INVALID_ARG for a missing pull source or arrived when pulling;
+ * CP_ERR_UNSUPPORTED when pulling with N > 64; CP_ERR_ALIGNMENT for a pull
+ * source not 16-byte or arrived not 4-byte aligned. A wait that runs out (2 s)
+ * ends the kernel with CP_ERR_TIMEOUT in cp_attn_check.
+ */
+CP_API int cp_attn_fwd_ring(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all,
+                            const void* const* pull_k, const void* const* pull_v, int* arrived,
+                            float* o_parts, float* lse_parts, cp_stream_t stream);
+
 /* Builds (and, with a device, uploads) the per-step schedules of one rank's ring
- * steps. Idempotent. Errors: CP_ERR_INVALID_ARG, CP_ERR_UNSUPPORTED (Ulysses),
+ * steps and of its one-launch forward. Idempotent. Errors: CP_ERR_INVALID_ARG, CP_ERR_UNSUPPORTED (Ulysses),
  * CP_ERR_CUDA (device allocation). */
 CP_API int cp_attn_ring_prepare(cp_attn_plan_t plan, int rank);
 
@@ -201,7 +239,9 @@ CP_API int cp_attn_ring_prepare(cp_attn_plan_t plan, int rank);
  * status; when items is not NULL writes n records of five int32 (row block
  * rank*B + b, head, query-tile pair, executed key tiles of the step, CTA) in
  * run order; when cta_loads is not NULL writes each CTA's modelled load (as
- * cp_attn_plan_cta_loads counts it; min(n, SM count) CTAs).
+ * cp_attn_plan_cta_loads counts it; min(n, SM count) CTAs). step = -1 gives
+ * the units of cp_attn_fwd_ring (N*B*H*pairs of them) with the query-tile pair
+ * field holding pair | (ring step << 16).
  */
 CP_API int64_t cp_attn_ring_schedule(cp_attn_plan_t plan, int rank, int step, int32_t* items,
                                      int64_t* cta_loads);

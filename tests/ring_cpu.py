@@ -1,104 +1,127 @@
 """A CPU model of one ring rank, for testing the ring protocol (``run_ring``)
 without a GPU.
 
-Each rank has two single-thread executors standing in for its compute and copy
-streams (work runs in submission order on each; a task may wait on another
-stream's future, like a stream waiting on an event), two receive slots holding a
-K/V block each, and a tag per slot naming the block it holds. Compute checks the
-tag of the slot it reads and computes the oracle partial; a pull checks the tag
-of the peer slot it copies before and after the copy (so a peer overwriting it
-mid-copy is caught) and sets its own slot's tag. Random sleeps in every task
-shake the interleavings.
+Each rank has a single-thread executor standing in for its stream and another
+for its copy stream, slot sets (set s, slot j: rank j's K/V block as fetched in a
+call that used set s; slot ``rank`` is filled with the rank's own block), and a
+tag per slot naming the (call, block) it holds. The forward runs as one task on
+the rank's stream, like the persistent kernel: a copier thread (the copy warps)
+fetches the other ranks' own blocks in ring order, checking each owner's slot tag
+before and after the copy (so a refill during the copy is caught), and raises a
+per-block arrival count; the units, step-major, wait (bounded) for their block's
+arrival, check the slot's tag and compute the oracle partial. The fill runs on
+the copy stream after everything on the rank's stream. Random sleeps shake the
+interleavings, and a rank can be given a slow copier, so that the others run
+ahead.
 """
 from __future__ import annotations
 
 import random
+import threading
 import time
 from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
-from context_long_sequence_cp_b200.ring import run_ring
+from context_long_sequence_cp_b200.ring import SLOT_SETS, run_ring
 from oracle.attention import merge, partial
 
 
 class CpuRank:
     def __init__(self, rank, N, q, k, v, qpos, pos_of, causal, scale, slots, tags, barrier, seed=0,
-                 jitter=0.002):
+                 jitter=0.002, pull_delay=0.0, sets=SLOT_SETS, fill_after_forward=True):
         """q, k, v: the rank's local [T, H, D] fp64 arrays; qpos [T] their global
         positions; pos_of(block) the positions of block ``block``'s tokens; slots
-        [2, 2, T, H, D] and tags [2] arrays of this rank (shared with the previous
-        rank); barrier() the host barrier."""
+        [sets, N, 2, T, H, D] and tags [sets, N] (int64) arrays of this rank,
+        readable by the other ranks; barrier() the host barrier."""
         self.rank, self.N = rank, N
         self.q, self.k, self.v, self.qpos, self.pos_of = q, k, v, qpos, pos_of
         self.causal, self.scale = causal, scale
         self.slots, self.tags, self.barrier = slots, tags, barrier
+        self.sets, self.fill_after_forward = sets, fill_after_forward
+        self.calls = 0
         self.rng = random.Random(seed * 1000 + rank)
         self.jitter = jitter
+        self.pull_delay = pull_delay      # extra time each fetched block takes (a slow link)
         self.errors = []
+        self.stream = ThreadPoolExecutor(1)
+        self.copy_stream = ThreadPoolExecutor(1)
+        self.last = None
 
     def _sleep(self):
         time.sleep(self.rng.random() * self.jitter)
 
-    def forward(self, next_slots, next_tags):
+    def close(self):
+        self.stream.shutdown(wait=True)
+        self.copy_stream.shutdown(wait=True)
+
+    def forward(self, peer_slots, peer_tags):
+        """peer_slots[j], peer_tags[j]: rank j's slot and tag arrays (own included).
+        Returns a future of (O, lse)."""
         N, r = self.N, self.rank
-        comp, copy = ThreadPoolExecutor(1), ThreadPoolExecutor(1)
-        parts = [None] * N
-        pull_done = [None] * max(N - 1, 1)
-        compute_done = [None] * N
+        c = self.calls
+        self.calls += 1
+        sset = c % self.sets
+        tag = lambda j: c * N + j
+        prev = self.last
 
         def fill_task():
+            if prev is not None and self.fill_after_forward:
+                prev.result()                     # stream order: after the previous forward
             self._sleep()
-            self.slots[0, 0] = self.k
-            self.slots[0, 1] = self.v
-            self.tags[0] = r
+            self.slots[sset, r, 0] = self.k
+            self.slots[sset, r, 1] = self.v
+            self.tags[sset, r] = tag(r)
 
-        fill_done = comp.submit(fill_task)
+        fill_done = []
 
-        def compute(t):
-            def task():
+        def forward_task():
+            arrived = np.zeros(N, dtype=np.int64)
+
+            def copier():
+                for t in range(1, N):
+                    j = (r + t) % N
+                    if int(peer_tags[j][sset, j]) != tag(j):
+                        self.errors.append(f"rank {r} call {c}: owner {j}'s slot holds {int(peer_tags[j][sset, j])}")
+                    buf = peer_slots[j][sset, j].copy()
+                    self._sleep()
+                    time.sleep(self.pull_delay)
+                    if int(peer_tags[j][sset, j]) != tag(j):
+                        self.errors.append(f"rank {r} call {c}: owner {j}'s slot refilled during the copy")
+                    self.slots[sset, j] = buf
+                    self.tags[sset, j] = tag(j)
+                    arrived[j] = 1
+
+            th = threading.Thread(target=copier)
+            th.start()
+            parts = []
+            T, H, D = self.q.shape
+            for t in range(N):
+                j = (r + t) % N
                 if t > 0:
-                    pull_done[t - 1].result()
-                self._sleep()
-                blk = (r + t) % N
-                if t == 0:
-                    kk, vv = self.k, self.v
-                else:
-                    if int(self.tags[t % 2]) != blk:
-                        self.errors.append(f"rank {r} step {t}: slot holds {int(self.tags[t % 2])}, wants {blk}")
-                    kk, vv = self.slots[t % 2, 0].copy(), self.slots[t % 2, 1].copy()
-                T, H, D = self.q.shape
+                    t0 = time.monotonic()
+                    while not arrived[j]:
+                        if time.monotonic() - t0 > 30:
+                            raise TimeoutError(f"rank {r}: block {j} never arrived")
+                        time.sleep(1e-4)
+                if int(self.tags[sset, j]) != tag(j):
+                    self.errors.append(f"rank {r} call {c} step {t}: slot {j} holds {int(self.tags[sset, j])}")
+                kk, vv = self.slots[sset, j, 0].copy(), self.slots[sset, j, 1].copy()
                 o = np.zeros((T, H, D))
                 lse = np.zeros((T, H))
                 for h in range(H):
-                    o[:, h], lse[:, h] = partial(self.q[:, h], self.qpos, kk[:, h], vv[:, h], self.pos_of(blk),
+                    o[:, h], lse[:, h] = partial(self.q[:, h], self.qpos, kk[:, h], vv[:, h], self.pos_of(j),
                                                  causal=self.causal, scale=self.scale)
-                parts[t] = (o.reshape(T * H, D), lse.reshape(T * H))
-            compute_done[t] = comp.submit(task)
+                parts.append((o.reshape(T * H, D), lse.reshape(T * H)))
+            th.join()
+            return merge(parts)
 
-        def pull(t):
-            def task():
-                fill_done.result()
-                if t >= 1:
-                    compute_done[t - 1].result()
-                want = (r + t + 1) % N
-                if int(next_tags[t % 2]) != want:
-                    self.errors.append(f"rank {r} pull {t}: peer slot holds {int(next_tags[t % 2])}, wants {want}")
-                buf = next_slots[t % 2].copy()
-                self._sleep()
-                if int(next_tags[t % 2]) != want:
-                    self.errors.append(f"rank {r} pull {t}: peer slot overwritten during the copy")
-                self.slots[(t + 1) % 2] = buf
-                self.tags[(t + 1) % 2] = want
-            pull_done[t] = copy.submit(task)
+        def fill():
+            fill_done.append(self.copy_stream.submit(fill_task))
 
-        try:
-            run_ring(N, compute, pull, wait_pull=lambda t: pull_done[t].result(),
-                     wait_compute=lambda t: compute_done[t].result(), barrier=self.barrier,
-                     wait_fill=fill_done.result)
-            for f in compute_done:
-                f.result()
-        finally:
-            comp.shutdown(wait=True)
-            copy.shutdown(wait=True)
-        return merge(parts)
+        def launch():
+            f = fill_done[0]
+            self.last = self.stream.submit(lambda: (f.result(), forward_task())[1])
+
+        run_ring(fill, lambda: fill_done[0].result(), self.barrier, launch)
+        return self.last

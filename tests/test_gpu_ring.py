@@ -2,11 +2,15 @@
 
 * ``cp_attn_fwd_ring_step``: every (rank, step) partial, computed from rank-local
   buffers, against the oracle's ring partial of that rank and step;
+* ``cp_attn_fwd_ring`` (a rank's N steps in one cooperative launch): bit-identical
+  to the N per-step launches (the same unit arithmetic), both on resident blocks
+  and when its copy warps fetch the other blocks themselves (the fetched slots
+  bit-identical to their sources); an arrival count that never fills ends the
+  kernel with CP_ERR_TIMEOUT and leaves the context usable;
 * the whole ring (``ring.RingRank``): N ranks emulated as host threads of one
-  process on one GPU, each with its own compute and copy streams, pulling the
-  next rank's slots by copy engine and meeting at a host barrier every step; each
-  rank's rows against the oracle's full attention, and against the fused
-  single-launch forward on the 4k zigzag workload;
+  process on one GPU (their launches on one stream), one host barrier per call,
+  calls back to back; each rank's rows against the oracle's full attention, and
+  against the fused single-launch forward on the 4k zigzag workload;
 * the IPC plumbing that can run in one process (handles, device views).
 The rank processes of a real multi-GPU ring need one GPU each; their protocol is
 checked on CPU with gloo processes (tests/test_ring_host.py).
@@ -62,14 +66,69 @@ def test_ring_step_matches_oracle_partials(B, H, S, D, N, layout, causal):
                 assert np.abs(lp[fin] - l_ref[fin]).max() <= G.TOL_LSE
 
 
+@pytest.mark.parametrize("B,H,S,D,N,layout,causal", [
+    (1, 2, 1024, 128, 4, "zigzag", True),
+    (2, 2, 1536, 64, 3, "contiguous", True),
+    (1, 3, 1920, 128, 5, "zigzag", True),
+])
+def test_ring_launch_equals_step_launches(B, H, S, D, N, layout, causal):
+    q, k, v = make_small(B, H, S, D, 80 + N)
+    plan = cp.Plan(B, H, S, D, N, causal, layout)
+    qd, kd, vd = (G.to_layout(x, N, layout).cuda() for x in (q, k, v))
+    arrived = torch.zeros(N, dtype=torch.int32, device="cuda")
+    for r in range(N):
+        op, lp = cp.attn_fwd_ring(plan, r, qd[r], kd, vd)                  # every block resident
+        # fused pull: only the own slot is filled; the copy warps fetch the rest
+        ks = torch.full_like(kd, float("nan"))
+        vs = torch.full_like(vd, float("nan"))
+        ks[r].copy_(kd[r])
+        vs[r].copy_(vd[r])
+        srcs_k = [kd[j].data_ptr() for j in range(N)]
+        srcs_v = [vd[j].data_ptr() for j in range(N)]
+        op2, lp2 = cp.attn_fwd_ring(plan, r, qd[r], ks, vs, srcs_k, srcs_v, arrived)
+        assert cp.check(plan) == 0
+        assert torch.equal(ks.view(torch.int16), kd.view(torch.int16))
+        assert torch.equal(vs.view(torch.int16), vd.view(torch.int16))
+        if N > 1:
+            chunks = -(-kd[0].numel() * 2 // 32768)
+            assert arrived.tolist() == [0 if j == r else 2 * chunks for j in range(N)]
+        for t in range(N):
+            rk = (r + t) % N
+            os_, ls_ = cp.attn_fwd_ring_step(plan, r, t, qd[r], kd[rk].contiguous(), vd[rk].contiguous())
+            assert torch.equal(op[t].view(torch.int32), os_.view(torch.int32)), (r, t)
+            assert torch.equal(lp[t].view(torch.int32), ls_.view(torch.int32)), (r, t)
+        assert torch.equal(op.view(torch.int32), op2.view(torch.int32))
+        assert torch.equal(lp.view(torch.int32), lp2.view(torch.int32))
+    assert cp.check(plan) == 0
+
+
+def test_ring_launch_times_out_on_a_block_that_never_arrives():
+    B, H, S, D, N = 1, 2, 1024, 128, 4
+    q, k, v = make_small(B, H, S, D, 90)
+    plan = cp.Plan(B, H, S, D, N, True, "zigzag")
+    qd, kd, vd = (G.to_layout(x, N, "zigzag").cuda() for x in (q, k, v))
+    arrived = torch.zeros(N, dtype=torch.int32, device="cuda")     # no pull, nothing raises the counts
+    cp.attn_fwd_ring(plan, 0, qd[0], kd, vd, arrived=arrived)
+    assert cp.check(plan) == -5                                    # CP_ERR_TIMEOUT, after the 2 s budget
+    assert cp.check(plan) == 0
+    # the context is still usable: the same launch with the blocks marked arrived
+    arrived.fill_(1)
+    op, lp = cp.attn_fwd_ring(plan, 0, qd[0], kd, vd, arrived=arrived)
+    assert cp.check(plan) == 0
+    os_, ls_ = cp.attn_fwd_ring_step(plan, 0, 2, qd[0], kd[2].contiguous(), vd[2].contiguous())
+    assert torch.equal(op[2].view(torch.int32), os_.view(torch.int32))
+
+
 def _run_ring(plan, qs, ks, vs, reps=1):
     ranks = R.thread_ring(plan)
     try:
+        outs = []
         for _ in range(reps):
             out = R.run_threads(ranks, list(zip(qs, ks, vs)))
+            outs.append([(o.clone(), l.clone()) for o, l in out])
         torch.cuda.synchronize()
         assert cp.check(plan) == 0
-        return [(o.clone(), l.clone()) for o, l in out]
+        return outs[-1]
     finally:
         for rr in ranks:
             rr.close()
@@ -86,7 +145,7 @@ def test_ring_threads_match_oracle(B, H, S, D, N, layout, causal):
     q, k, v = make_small(B, H, S, D, 70 + N)
     plan = cp.Plan(B, H, S, D, N, causal, layout)
     qs, ks, vs = (_rank_inputs(x, N, layout) for x in (q, k, v))
-    out = _run_ring(plan, qs, ks, vs, reps=2)       # the second call reuses the slots
+    out = _run_ring(plan, qs, ks, vs, reps=3)       # calls alternate between the two slot sets
     f = lambda t: t.float().numpy()
     o_ref, lse_ref = A.attention(f(q), f(k), f(v), causal=causal)       # [B, S, H, D], [B, H, S]
     pos = L.chunk_positions(S, N, layout)

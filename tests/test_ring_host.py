@@ -1,12 +1,15 @@
-"""Host-side checks of the multi-GPU ring (no GPU): the per-rank step schedules
-of the C library, and the ring protocol (``run_ring``) on a CPU model of the
-ranks' streams, as threads of one process and as gloo processes.
+"""Host-side checks of the multi-GPU ring (no GPU): the per-rank schedules of
+the C library (per ring step, and the one-launch forward's units), and the ring
+protocol (``run_ring``) on a CPU model of the ranks' streams and copy warps, as
+threads of one process and as gloo processes.
 
-The protocol runs each rank on its own block first, pulls block (r + t + 1) mod N
-from rank r + 1 while step t computes, and orders the ranks by host barriers
-(page "序列与上下文并行", section "上下文并行：注意力本身切分": the K/V blocks
-travel around the ring while each rank computes on the one it holds). The
-result must equal full attention for every rank's rows (oracle).
+The protocol fills each rank's own slot, meets the other ranks at one barrier,
+and runs the forward, which fetches the other ranks' own blocks in ring order
+while it computes (page "序列与上下文并行", section "上下文并行：注意力本身切分":
+each rank computes on the blocks it holds while the next ones arrive). Calls
+run back to back, alternating between two slot sets. The result must equal full
+attention for every rank's rows (oracle), and no fetch may read a slot before
+its owner filled it or while its owner refills it.
 """
 import ctypes
 import os
@@ -103,17 +106,56 @@ def test_ring_schedule_balance_zigzag_32k():
                 assert loads.sum() == 256 * (2 * 32 + 3) + 256 * 3 or loads.sum() == 512 * (2 * 16 + 3)
 
 
+@pytest.mark.parametrize("S,N,layout,causal,B,H", [(4096, 4, "zigzag", True, 1, 4), (2048, 4, "contiguous", True, 2, 2),
+                                                     (3840, 5, "zigzag", True, 1, 2)])
+def test_ring_launch_units_cover_every_step_once(S, N, layout, causal, B, H):
+    p = cp.Plan(B, H, S, 128, N, causal, layout)
+    npairs = -(-(S // N) // 256)
+    for r in range(N):
+        units, loads = p.ring_schedule(r, -1)
+        assert len(units) == N * B * H * npairs
+        seen = {(qp >> 16, rb, h, qp & 0xffff) for rb, h, qp, _, _ in units}
+        assert seen == {(t, r * B + b, h, qp) for t in range(N) for b in range(B) for h in range(H)
+                        for qp in range(npairs)}
+        walks = {t: _step_walk_lengths(S, N, layout, causal, r, t) for t in range(N)}
+        for rb, h, qp, cost, cta in units:
+            assert cost == walks[qp >> 16][qp & 0xffff]
+        # each CTA's units run in step order; CTAs are contiguous runs
+        assert [u[4] for u in units] == sorted(u[4] for u in units)
+        for c in set(u[4] for u in units):
+            steps = [u[2] >> 16 for u in units if u[4] == c]
+            assert steps == sorted(steps)
+        assert sum(loads) == sum(2 * u[3] + 3 for u in units)
+        assert max(loads) <= np.mean(loads) + max(2 * u[3] + 3 for u in units)
+
+
 def test_ring_argument_validation():
     p = cp.Plan(1, 2, 1024, 64, 4, True, "zigzag")
     L = cp.lib()
+    buf = ctypes.c_void_p(16)
     assert L.cp_attn_ring_prepare(None, 0) == -1
     assert L.cp_attn_ring_prepare(p.handle, -1) == -1
     assert L.cp_attn_ring_prepare(p.handle, 4) == -1
     assert L.cp_attn_ring_prepare(p.handle, 3) == 0           # host schedules only without a device
     assert L.cp_attn_ring_schedule(p.handle, 0, 4, None, None) == -1
+    assert L.cp_attn_ring_schedule(p.handle, 0, -2, None, None) == -1
+    assert L.cp_attn_ring_schedule(p.handle, 2, -1, None, None) == 4 * 2   # all steps' units
+    srcs = ctypes.cast((ctypes.c_void_p * 4)(16, 32, 48, 64), ctypes.c_void_p)
+    bad_src = ctypes.cast((ctypes.c_void_p * 4)(16, 40, 48, 64), ctypes.c_void_p)
+    null_src = ctypes.cast((ctypes.c_void_p * 4)(16, None, 48, 64), ctypes.c_void_p)
+    ring = lambda *a: L.cp_attn_fwd_ring(p.handle, *a)
+    assert ring(0, None, buf, buf, None, None, None, buf, buf, None) == -1
+    assert ring(5, buf, buf, buf, None, None, None, buf, buf, None) == -1
+    assert ring(0, buf, buf, buf, srcs, None, buf, buf, buf, None) == -1          # K sources without V
+    assert ring(0, buf, buf, buf, srcs, srcs, None, buf, buf, None) == -1         # pulling needs arrived
+    assert ring(0, buf, buf, buf, null_src, srcs, buf, buf, buf, None) == -1      # a missing source
+    assert ring(0, buf, buf, buf, bad_src, srcs, buf, buf, buf, None) == -3       # a misaligned source
+    assert ring(0, buf, buf, buf, None, None, ctypes.c_void_p(18), buf, buf, None) == -3
+    big = cp.Plan(1, 2, 65 * 256, 64, 65, False, "contiguous")
+    srcs65 = ctypes.cast((ctypes.c_void_p * 65)(*([16] * 65)), ctypes.c_void_p)
+    assert L.cp_attn_fwd_ring(big.handle, 0, buf, buf, buf, srcs65, srcs65, buf, buf, buf, None) == -2
     assert L.cp_attn_ring_schedule(p.handle, 4, 0, None, None) == -1
     assert L.cp_attn_ring_schedule(p.handle, 1, 2, None, None) == 2   # 2 heads x 1 query-tile pair (T = 256)
-    buf = ctypes.c_void_p(16)
     assert L.cp_attn_fwd_ring_step(p.handle, 0, 0, None, buf, buf, buf, buf, None) == -1
     assert L.cp_attn_fwd_ring_step(p.handle, 4, 0, buf, buf, buf, buf, buf, None) == -1
     assert L.cp_attn_fwd_ring_step(p.handle, 0, -1, buf, buf, buf, buf, buf, None) == -1
@@ -121,6 +163,7 @@ def test_ring_argument_validation():
     u = cp.Plan(1, 4, 1024, 64, 2, False, "ulysses")
     assert L.cp_attn_ring_prepare(u.handle, 0) == -2
     assert L.cp_attn_fwd_ring_step(u.handle, 0, 0, buf, buf, buf, buf, buf, None) == -2
+    assert L.cp_attn_fwd_ring(u.handle, 0, buf, buf, buf, None, None, None, buf, buf, None) == -2
     assert L.cp_ipc_handle_bytes() == 64
     assert L.cp_ipc_get_handle(None, ctypes.create_string_buffer(64)) == -1
     assert L.cp_copy_async(None, None, 0, None) == 0
@@ -147,38 +190,64 @@ def _check_rank(r, o, lse, pos, o_ref, lse_ref, H, D):
     np.testing.assert_allclose(lse.reshape(T, H), lse_ref[:, pos[r]].T, atol=1e-12, rtol=0)
 
 
-@pytest.mark.parametrize("N,layout,causal", [(1, "zigzag", True), (2, "zigzag", True), (3, "contiguous", True),
-                                             (4, "zigzag", True), (5, "contiguous", False)])
-def test_ring_protocol_threads(N, layout, causal):
+def _thread_ring(N, layout, causal, sets=None, fill_after_forward=True, calls=3, slow_rank=0):
     from tests.ring_cpu import CpuRank
+    from context_long_sequence_cp_b200.ring import SLOT_SETS
+    sets = SLOT_SETS if sets is None else sets
     H, D = 2, 8
     S, q, k, v, pos, o_ref, lse_ref = _problem(N, layout, causal, seed=N)
     T = S // N
     bar = threading.Barrier(N, timeout=60)
-    slots = [np.zeros((2, 2, T, H, D)) for _ in range(N)]
-    tags = [np.full(2, -1, dtype=np.int64) for _ in range(N)]
+    slots = [np.zeros((sets, N, 2, T, H, D)) for _ in range(N)]
+    tags = [np.full((sets, N), -1, dtype=np.int64) for _ in range(N)]
+    # one rank fetches slowly: the others run ahead into the next calls and would
+    # refill their slots under its fetches if the protocol let them
     ranks = [CpuRank(r, N, q[pos[r]], k[pos[r]], v[pos[r]], pos[r], lambda b: pos[b], causal, default_scale(D),
-                     slots[r], tags[r], bar.wait, seed=N) for r in range(N)]
-    for rep in range(2):                       # a second call reuses the slots
-        out = [None] * N
-        errs = []
+                     slots[r], tags[r], bar.wait, seed=N, pull_delay=0.01 if r == slow_rank else 0.0, sets=sets,
+                     fill_after_forward=fill_after_forward) for r in range(N)]
+    outs = [[] for _ in range(N)]
+    errs = []
 
-        def body(r):
+    def body(r):
+        try:
+            futs = [ranks[r].forward(slots, tags) for _ in range(calls)]
+            outs[r] = [f.result(timeout=60) for f in futs]
+        except BaseException as e:  # noqa: BLE001
+            errs.append(e)
+            bar.abort()
+
+    th = [threading.Thread(target=body, args=(r,)) for r in range(N)]
+    for t_ in th:
+        t_.start()
+    for t_ in th:
+        t_.join(120)
+    for rr in ranks:
+        rr.close()
+    bad = []
+    for r in range(N):
+        bad += ranks[r].errors
+        for o, lse in outs[r]:
             try:
-                out[r] = ranks[r].forward(slots[(r + 1) % N], tags[(r + 1) % N])
-            except BaseException as e:  # noqa: BLE001
-                errs.append(e)
-                bar.abort()
+                _check_rank(r, o, lse, pos, o_ref, lse_ref, H, D)
+            except AssertionError:
+                bad.append(f"rank {r}: wrong result")
+    return errs, bad
 
-        th = [threading.Thread(target=body, args=(r,)) for r in range(N)]
-        for t_ in th:
-            t_.start()
-        for t_ in th:
-            t_.join(120)
-        assert not errs, errs
-        for r in range(N):
-            assert not ranks[r].errors, ranks[r].errors
-            _check_rank(r, *out[r], pos, o_ref, lse_ref, H, D)
+
+@pytest.mark.parametrize("N,layout,causal", [(1, "zigzag", True), (2, "zigzag", True), (3, "contiguous", True),
+                                             (4, "zigzag", True), (5, "contiguous", False)])
+def test_ring_protocol_threads(N, layout, causal):
+    errs, bad = _thread_ring(N, layout, causal)
+    assert not errs, errs
+    assert not bad, bad
+
+
+def test_ring_protocol_checks_catch_a_reused_slot_set():
+    # One slot set and a fill not ordered after the rank's previous forward: a
+    # fast rank refills its block while the slow rank still fetches it. The
+    # model must notice (this is what the two alternating sets prevent).
+    errs, bad = _thread_ring(4, "zigzag", True, sets=1, fill_after_forward=False, calls=3, slow_rank=0)
+    assert errs or bad
 
 
 def _free_port():
@@ -201,30 +270,38 @@ def _gloo_worker(rank, world, port, prefix, layout, causal, q_out):
         H, D = 2, 8
         S, q, k, v, pos, o_ref, lse_ref = _problem(world, layout, causal, seed=7)
         T = S // world
-        shape = (2, 2, T, H, D)
-        nbytes = int(np.prod(shape)) * 8 + 16
+        from context_long_sequence_cp_b200.ring import SLOT_SETS
+        shape = (SLOT_SETS, world, 2, T, H, D)
+        nbytes = int(np.prod(shape)) * 8 + 8 * SLOT_SETS * world
         own = shared_memory.SharedMemory(name=f"{prefix}_{rank}", create=True, size=nbytes)
         shms.append(own)
         dist.barrier()
-        peer = shared_memory.SharedMemory(name=f"{prefix}_{(rank + 1) % world}")
-        shms.append(peer)
-        view = lambda m: (np.ndarray(shape, np.float64, m.buf, 16), np.ndarray(2, np.int64, m.buf, 0))
+        view = lambda m: (np.ndarray(shape, np.float64, m.buf, 8 * SLOT_SETS * world),
+                          np.ndarray((SLOT_SETS, world), np.int64, m.buf, 0))
+        peers = {j: shared_memory.SharedMemory(name=f"{prefix}_{j}") for j in range(world) if j != rank}
+        shms.extend(peers.values())
         slots, tags = view(own)
         tags[:] = -1
-        nslots, ntags = view(peer)
+        all_slots, all_tags = [], []
+        for j in range(world):
+            sj, tj = (slots, tags) if j == rank else view(peers[j])
+            all_slots.append(sj)
+            all_tags.append(tj)
         dist.barrier()
         rr = CpuRank(rank, world, q[pos[rank]], k[pos[rank]], v[pos[rank]], pos[rank], lambda b: pos[b], causal,
-                     default_scale(D), slots, tags, dist.barrier, seed=11)
+                     default_scale(D), slots, tags, dist.barrier, seed=11, pull_delay=0.01 if rank == 0 else 0.0)
         ok = True
-        for _ in range(2):
-            o, lse = rr.forward(nslots, ntags)
+        futs = [rr.forward(all_slots, all_tags) for _ in range(3)]
+        for f in futs:
+            o, lse = f.result(timeout=60)
             try:
                 _check_rank(rank, o, lse, pos, o_ref, lse_ref, H, D)
             except AssertionError:
                 ok = False
+        rr.close()
         dist.barrier()
         q_out.put((rank, ok, list(rr.errors)))
-        del slots, tags, nslots, ntags
+        del rr, slots, tags, all_slots, all_tags, sj, tj   # release the views before closing the segments
     finally:
         for m in shms:
             m.close()
