@@ -433,17 +433,20 @@ def main():
         cp.attn_fwd_ring(plan, 0, q0, kz, vz, o_parts=op_r, lse_parts=lp_r, stream=stream)
         cp.merge_partials(op_r, lp_r, o_out=ro, lse_out=rl)
 
+    op_s = torch.empty(N, plan.rows // N, D, dtype=torch.float32, device=dev)
+    lp_s = torch.empty(N, plan.rows // N, dtype=torch.float32, device=dev)
+
     def step_launches():
         for t in range(N):
-            cp.attn_fwd_ring_step(plan, 0, t, q0, kz[t], vz[t], op_r[t], lp_r[t], stream)
-        cp.merge_partials(op_r, lp_r, o_out=ro, lse_out=rl)
+            cp.attn_fwd_ring_step(plan, 0, t, q0, kz[t], vz[t], op_s[t], lp_s[t], stream)
+        cp.merge_partials(op_s, lp_s, o_out=ro, lse_out=rl)
 
     ring_launch_ms = time_flushed(launch_only)
     ring_steps_ms = time_flushed(step_launches)
     if cp.check(plan) != 0:
         raise RuntimeError("ring runs failed")
     rr.close()
-    del l2_flush
+    del l2_flush, op_s, lp_s
 
     # --- end to end through the public API from pinned host buffers. Every step
     # uploads its own Q/K/V from pinned memory and reads back its own O and lse;
@@ -557,9 +560,11 @@ def main():
             "ring_overhead_vs_fused_share": ring_ms / (att / N) - 1.0,
             "ring_fetch_cost": ring_ms / ring_launch_ms - 1.0,
             "ring_fetch_bytes": (N - 1) * 2 * blk,
+            "ring_parts": plan.ring_parts(),
             "ring_note": f"rank 0 of {N} on one GPU: fill + one cooperative launch whose copy warps fetch the "
                          f"other {N - 1} K/V blocks ({(N - 1) * 2 * blk >> 20} MiB; here from local HBM, on N "
-                         "GPUs over NVLink) while its units compute, + merge; launch_only = blocks resident; "
+                         "GPUs over NVLink) while its units compute (first half of the steps one unit per step, "
+                         "then one unit per query pair), + merge of the parts; launch_only = blocks resident; "
                          "step_launches = one launch per ring step; fused_share = the fused launch / N",
         },
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

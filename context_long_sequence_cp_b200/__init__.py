@@ -49,6 +49,7 @@ SIGNATURES = {
     "cp_attn_fwd_ulysses_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P]),
     "cp_attn_fwd_ring_step": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _P]),
     "cp_attn_ring_prepare": (_I, [_P, _I]),
+    "cp_attn_ring_num_parts": (_I, [_P]),
     "cp_attn_fwd_ring": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "cp_attn_ring_schedule": (_I64, [_P, _I, _I, _P, _P]),
     "cp_ring_buffer_alloc": (_I, [_SZ, ctypes.POINTER(_P)]),
@@ -167,10 +168,18 @@ class Plan:
         """Build (and upload) the per-step schedules of one rank's ring steps."""
         _check("cp_attn_ring_prepare", lib().cp_attn_ring_prepare(self._h, int(rank)))
 
+    def ring_parts(self) -> int:
+        """Number of partials of the one-launch ring forward."""
+        n = int(lib().cp_attn_ring_num_parts(self._h))
+        if n < 0:
+            raise CpAttnError("cp_attn_ring_num_parts", n)
+        return n
+
     def ring_schedule(self, rank: int, step: int):
         """Schedule of one rank's ring step: (items as rows of (row block, head,
         query-tile pair, key tiles, CTA) in run order, per-CTA modelled loads);
-        step -1: the units of the one-launch ring forward (pair | step << 16)."""
+        step -1: the units of the one-launch ring forward (pair | first step << 16 |
+    end step << 24)."""
         n = int(lib().cp_attn_ring_schedule(self._h, int(rank), int(step), None, None))
         if n < 0:
             raise CpAttnError("cp_attn_ring_schedule", n)
@@ -242,12 +251,14 @@ def attn_fwd_ring(plan: Plan, rank: int, q, k_all, v_all, pull_k=None, pull_v=No
     j's block; slot ``rank`` filled). pull_k, pull_v: N device addresses of the
     ranks' own blocks to fetch from (None: every slot already filled). arrived:
     int32 [N] device tensor (needed when pulling). Returns (o_parts fp32
-    [N, rows, D], lse_parts fp32 [N, rows]), rows = B*(S/N)*H."""
+    [P, rows, D], lse_parts fp32 [P, rows]), P = plan.ring_parts(),
+    rows = B*(S/N)*H."""
     rows = plan.B * (plan.S // plan.N) * plan.H
+    P = plan.ring_parts()
     if o_parts is None:
-        o_parts = torch.empty(plan.N, rows, plan.D, dtype=torch.float32, device=q.device)
+        o_parts = torch.empty(P, rows, plan.D, dtype=torch.float32, device=q.device)
     if lse_parts is None:
-        lse_parts = torch.empty(plan.N, rows, dtype=torch.float32, device=q.device)
+        lse_parts = torch.empty(P, rows, dtype=torch.float32, device=q.device)
     pk = None if pull_k is None else (ctypes.c_void_p * len(pull_k))(*[int(x) for x in pull_k])
     pv = None if pull_v is None else (ctypes.c_void_p * len(pull_v))(*[int(x) for x in pull_v])
     as_ptr = lambda a: None if a is None else ctypes.cast(a, ctypes.c_void_p)

@@ -277,6 +277,10 @@ int ensure_device(cp_attn_plan_s* p) {
   return CP_ERR_CUDA;
 }
 
+// First step of the tail phase of a one-launch ring forward: half the steps run
+// one unit per step, the rest in one unit per query-tile pair.
+int ring_split(int nr) { return nr <= 2 ? nr : (nr + 1) / 2; }
+
 // Schedules of one rank's ring steps: at step t the rank's items (every batch,
 // head and query-tile pair) carry the key tiles of their walk at step t, and are
 // assigned to CTAs by the whole-view list's greedy rule, longest first.
@@ -312,32 +316,51 @@ void build_ring_rank(cp_attn_plan_s* p, int r) {
     std::copy(load.begin(), load.end(), rr.cta_load.begin() + static_cast<size_t>(t) * p->sms);
     rr.items.insert(rr.items.end(), items.begin(), items.end());
   }
-  // One launch over all steps: the units of step t follow those of step t - 1,
-  // so that the CTAs reach a block in about the order the blocks arrive.
-  std::vector<WorkItem> units;
-  std::vector<int64_t> cost;
-  units.reserve(rr.items.size());
-  cost.reserve(rr.items.size());
-  for (int t = 0; t < g.NR; ++t)
-    for (int i = 0; i < rr.nper; ++i) {
-      WorkItem w = rr.items[static_cast<size_t>(t) * rr.nper + i];
-      cost.push_back(2 * static_cast<int64_t>(w.cost) + kItemOverheadHalfTiles);
-      w.qp = pack_unit_qp(w.qp, t);
-      units.push_back(w);
+  // One launch over all steps, in two phases. Steps [0, split) run as one unit
+  // per (step, pair), step-major, while the later blocks are still arriving;
+  // then each pair walks steps [split, NR) in one unit, its softmax state kept
+  // on chip as in the fused kernel. split + 1 partials (NR when split = NR - 1).
+  rr.units.clear();
+  rr.unit_cta_begin.assign(1, 0);
+  rr.unit_cta_load.clear();
+  rr.unit_n_cta = 0;
+  if (g.NR > 255) {   // unit steps are packed in 8 bits: no one-launch schedule
+    rr.built = true;
+    return;
+  }
+  const int split = ring_split(g.NR);
+  struct U {
+    WorkItem w;
+    int64_t cost;
+    int phase;   // the step for the first phase, split for the tail
+  };
+  std::vector<U> us;
+  us.reserve(static_cast<size_t>(rr.nper) * (split + 1));
+  for (int b = 0; b < g.B; ++b)
+    for (int qp = 0; qp < p->npairs; ++qp) {
+      const int* off = p->step_off.data() + static_cast<size_t>(r * p->npairs + qp) * (g.NR + 1);
+      for (int h = 0; h < g.Hh; ++h) {
+        for (int t = 0; t < split; ++t) {
+          const int len = off[t + 1] - off[t];
+          us.push_back(U{WorkItem{r * g.B + b, h, pack_unit(qp, t, t + 1), len},
+                         2 * static_cast<int64_t>(len) + kItemOverheadHalfTiles, t});
+        }
+        if (split < g.NR) {
+          const int len = off[g.NR] - off[split];
+          us.push_back(U{WorkItem{r * g.B + b, h, pack_unit(qp, split, g.NR), len},
+                         2 * static_cast<int64_t>(len) + kItemOverheadHalfTiles, split});
+        }
+      }
     }
-  // rr.items is grouped by CTA within each step; restore the longest-first order
-  std::vector<size_t> order(units.size());
-  for (size_t i = 0; i < order.size(); ++i) order[i] = i;
-  std::stable_sort(order.begin(), order.end(), [&](size_t a, size_t b) {
-    const int ta = item_step(units[a]), tb = item_step(units[b]);
-    if (ta != tb) return ta < tb;
-    return cost[a] > cost[b];
+  std::stable_sort(us.begin(), us.end(), [](const U& x, const U& y) {
+    if (x.phase != y.phase) return x.phase < y.phase;
+    return x.cost > y.cost;
   });
   rr.units.clear();
   std::vector<int64_t> ucost;
-  for (size_t i : order) {
-    rr.units.push_back(units[i]);
-    ucost.push_back(cost[i]);
+  for (const U& u : us) {
+    rr.units.push_back(u.w);
+    ucost.push_back(u.cost);
   }
   rr.unit_n_cta = assign_greedy(rr.units, ucost, p->sms, rr.unit_cta_begin, rr.unit_cta_load);
   rr.built = true;
@@ -356,12 +379,14 @@ void free_ring(cp_attn_plan_s::RingRank& rr) {
 int upload_ring_rank(cp_attn_plan_s::RingRank& rr) {
   if (rr.d_items != nullptr) return CP_OK;
   const size_t ib = rr.items.size() * sizeof(WorkItem), cb = rr.cta_begin.size() * sizeof(int);
-  const size_t ub = rr.units.size() * sizeof(WorkItem), ucb = rr.unit_cta_begin.size() * sizeof(int);
+  const size_t ub = (rr.units.empty() ? 1 : rr.units.size()) * sizeof(WorkItem);
+  const size_t ucb = rr.unit_cta_begin.size() * sizeof(int);
   const bool ok = cudaMalloc(&rr.d_items, ib) == cudaSuccess && cudaMalloc(&rr.d_cta_begin, cb) == cudaSuccess &&
                   cudaMalloc(&rr.d_units, ub) == cudaSuccess && cudaMalloc(&rr.d_unit_cta_begin, ucb) == cudaSuccess &&
                   cudaMemcpy(rr.d_items, rr.items.data(), ib, cudaMemcpyHostToDevice) == cudaSuccess &&
                   cudaMemcpy(rr.d_cta_begin, rr.cta_begin.data(), cb, cudaMemcpyHostToDevice) == cudaSuccess &&
-                  cudaMemcpy(rr.d_units, rr.units.data(), ub, cudaMemcpyHostToDevice) == cudaSuccess &&
+                  (rr.units.empty() ||
+                   cudaMemcpy(rr.d_units, rr.units.data(), ub, cudaMemcpyHostToDevice) == cudaSuccess) &&
                   cudaMemcpy(rr.d_unit_cta_begin, rr.unit_cta_begin.data(), ucb, cudaMemcpyHostToDevice) ==
                       cudaSuccess;
   if (!ok) {
@@ -741,6 +766,13 @@ int cp_attn_ring_prepare(cp_attn_plan_t plan, int rank) {
   return upload_ring_rank(rr);
 }
 
+int cp_attn_ring_num_parts(cp_attn_plan_t plan) {
+  if (plan == nullptr) return CP_ERR_INVALID_ARG;
+  if (plan->layout == CP_LAYOUT_ULYSSES) return CP_ERR_UNSUPPORTED;
+  const int split = ring_split(plan->N);
+  return split < plan->N ? split + 1 : plan->N;
+}
+
 int64_t cp_attn_ring_schedule(cp_attn_plan_t plan, int rank, int step, int32_t* items, int64_t* cta_loads) {
   if (plan == nullptr) return CP_ERR_INVALID_ARG;
   if (plan->layout == CP_LAYOUT_ULYSSES) return CP_ERR_UNSUPPORTED;
@@ -833,6 +865,7 @@ int cp_attn_fwd_ring(cp_attn_plan_t plan, int rank, const void* q, void* k_all, 
   const bool pull = pull_k != nullptr && plan->N > 1;
   if (pull && arrived == nullptr) return CP_ERR_INVALID_ARG;
   if (pull && plan->N > kMaxPullRanks) return CP_ERR_UNSUPPORTED;
+  if (plan->N > 255) return CP_ERR_UNSUPPORTED;   // unit steps are packed in 8 bits
   if (!aligned16(q) || !aligned16(k_all) || !aligned16(v_all) || !aligned16(o_parts) || !aligned16(lse_parts) ||
       (reinterpret_cast<uintptr_t>(arrived) & 3u))
     return CP_ERR_ALIGNMENT;
@@ -881,6 +914,7 @@ int cp_attn_fwd_ring(cp_attn_plan_t plan, int rank, const void* q, void* k_all, 
   P.q_rb0 = rank * g.B;
   P.kv_local = 0;
   P.unit_steps = 1;
+  P.unit_split = ring_split(g.NR);
   P.part_rows = static_cast<int64_t>(g.B) * g.T * g.Hh;
   P.arrived = arrived;
   P.arrive_target = pull ? P.pull_chunks : 1;

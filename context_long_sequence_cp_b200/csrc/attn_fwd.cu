@@ -181,8 +181,8 @@ __device__ __forceinline__ void item_walk(const FwdParams& p, const WorkItem& w,
   const int* off = p.step_off + (rq * p.npairs + qp) * (p.g.NR + 1);
   int t0 = p.t_begin, t1 = p.t_end;
   if (PARTIAL && p.unit_steps) {
-    t0 = item_step(w);
-    t1 = t0 + 1;
+    t0 = unit_t0(w);
+    t1 = unit_t1(w);
   }
   e_begin = __ldg(off + t0);
   e_end = __ldg(off + t1);
@@ -252,13 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q0 = (PARTIAL ? item_qp(w) : w.qp) * kPair;
         int e_begin, e_end;
         item_walk<PARTIAL>(p, w, rq, e_begin, e_end);
-        if (PARTIAL && p.arrived != nullptr && e_begin < e_end) {
-          // another rank's block: wait until all of it has arrived
-          const int rk = entry_rank(__ldg(p.entries + e_begin));
-          if (rk != rq) ok = count_wait(p.arrived + rk, p.arrive_target, ctl);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-        }
         if (q_iter > 0) ok = mbar_wait(smem_addr(&sm.q_empty), (q_iter - 1) & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
@@ -269,8 +262,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d_elect(smem_addr(&sm.q[i][0]) + blk * C::kBlockBytes, &tm_q, qbar, blk * 64, w.h,
                         q0 + i * kTile, w.rb - p.q_rb0, pol_q);
         ++q_iter;
+        int waited = rq;   // the block last waited for (the own block needs no wait)
         for (int e = e_begin; e < e_end && ok; ++e) {
           const uint32_t ent = __ldg(p.entries + e);
+          if (PARTIAL && p.arrived != nullptr && entry_rank(ent) != waited) {
+            // first load from another rank's block: wait until all of it has arrived
+            waited = entry_rank(ent);
+            ok = count_wait(p.arrived + waited, p.arrive_target, ctl);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+          }
           const int rbk = p.kv_local ? bv : entry_rank(ent) * g.B + bv;
           const int k0 = entry_tile(ent) * kTile;
           for (int which = 0; which < 2; ++which) {
@@ -542,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int bv = w.rb % g.B;
       const int tl = (PARTIAL ? item_qp(w) : w.qp) * kPair + wg * kTile + row;
       const int64_t row_id = (static_cast<int64_t>(w.rb - p.q_rb0) * g.T + tl) * g.Hh + w.h +
-                             (PARTIAL && p.unit_steps ? item_step(w) * p.part_rows : 0);
+                             (PARTIAL && p.unit_steps ? min(unit_t0(w), p.unit_split) * p.part_rows : 0);
       if (ntile > 0) {
         ok = mbar_wait(smem_addr(&sm.o_done[wg]), od_cnt & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);

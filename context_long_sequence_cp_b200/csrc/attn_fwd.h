@@ -37,11 +37,13 @@ struct FwdParams {
   // v maps hold the key rank's B row blocks only.
   int q_rb0;
   int kv_local;
-  // Ring launches (partial mode): every item is a (ring step, item) unit whose
-  // partial goes to part item_step(w), part_rows rows per part; before reading
+  // Ring launches (partial mode): every item is a unit, a query-tile pair over
+  // ring steps [unit_t0, unit_t1), whose partial goes to part
+  // min(unit_t0, unit_split), part_rows rows per part; before its first load from
   // the key/value block of another rank k the producer waits until arrived[k]
   // >= arrive_target (arrived null: no wait).
   int unit_steps;
+  int unit_split;
   int64_t part_rows;
   int* arrived;
   int arrive_target;

@@ -91,11 +91,16 @@ struct WorkItem {
   int cost;  // executed key tiles (both query tiles), used for ordering
 };
 
-// Ring launches run one rank's (ring step, item) units, the step in the high
-// half of qp; everywhere else the high half is zero.
+// Ring launches run one rank's units: a query-tile pair over ring steps
+// [t0, t1), packed as qp | t0 << 16 | t1 << 24 (steps < 256); everywhere else
+// the high half of qp is zero.
 CP_HD int item_qp(const WorkItem& w) { return w.qp & 0xffff; }
-CP_HD int item_step(const WorkItem& w) { return static_cast<int>(static_cast<unsigned>(w.qp) >> 16); }
-CP_HD int pack_unit_qp(int qp, int step) { return qp | (step << 16); }
+CP_HD int unit_t0(const WorkItem& w) { return static_cast<int>((static_cast<unsigned>(w.qp) >> 16) & 0xffu); }
+CP_HD int unit_t1(const WorkItem& w) { return static_cast<int>(static_cast<unsigned>(w.qp) >> 24); }
+CP_HD int pack_unit(int qp, int t0, int t1) {
+  return static_cast<int>(static_cast<unsigned>(qp) | (static_cast<unsigned>(t0) << 16) |
+                          (static_cast<unsigned>(t1) << 24));
+}
 
 // A precomputed key-tile entry of a work item's walk, packed in 32 bits:
 // bits [0,13) key tile index, [13,25) key rank, [25,27) class of query tile 0,

@@ -11,10 +11,12 @@ bandwidth, so rank r fetches block (r + t) mod N straight from its owner rather
 than having it relayed hop by hop: the same bytes per rank (N - 1 blocks), no
 chain of per-step hand-offs. Each rank exposes its own block in a slot buffer
 the others map through CUDA IPC. The whole forward is ONE persistent,
-cooperative kernel launch (``cp_attn_fwd_ring``): its units run step-major,
-starting on the rank's own block, while two copy warps of every CTA load the
-other blocks over NVLink, in ring order, into local slots, publishing per-block
-arrival counts that the units wait on. The transfer overlaps the math inside one
+cooperative kernel launch (``cp_attn_fwd_ring``): the first half of the ring
+steps runs step-major, one unit per (step, query-tile pair), starting on the
+rank's own block; then each pair walks the remaining steps in one unit. Two
+copy warps of every CTA meanwhile load the other blocks over NVLink, in ring
+order, into local slots, publishing per-block arrival counts that the units
+wait on. The transfer overlaps the math inside one
 kernel and needs no copy engine, stream or event between them (a device-to-device
 copy issued on another stream does not progress while the persistent kernel
 holds every SM). The ranks meet at ONE host barrier per call, after every rank's
@@ -83,8 +85,9 @@ class RingRank:
         self.slots = DeviceBuffer(SLOT_SETS * self.set_bytes)
         self.peer_bases: Optional[list] = None
         self.arrived = torch.zeros(N, dtype=torch.int32, device=self.device)
-        self.o_parts = torch.empty(N, self.rows, D, dtype=torch.float32, device=self.device)
-        self.lse_parts = torch.empty(N, self.rows, dtype=torch.float32, device=self.device)
+        P = plan.ring_parts()
+        self.o_parts = torch.empty(P, self.rows, D, dtype=torch.float32, device=self.device)
+        self.lse_parts = torch.empty(P, self.rows, dtype=torch.float32, device=self.device)
         self.calls = 0
         self.copy_stream = torch.cuda.Stream(device=self.device)
         self.fill_done = torch.cuda.Event()

@@ -193,9 +193,13 @@ CP_API int cp_attn_fwd_ring_step(cp_attn_plan_t plan, int rank, int step, const 
 /*
  * One rank's whole ring forward in one launch, fetching the other ranks' blocks
  * itself. Page "序列与上下文并行", section "上下文并行：注意力本身切分": the rank
- * computes on the blocks it holds while the next ones arrive. The units (ring
- * step, pair of query tiles) run step-major on persistent CTAs, starting on the
- * rank's own block; meanwhile two copy warps of every CTA fetch the blocks of
+ * computes on the blocks it holds while the next ones arrive. The work runs on
+ * persistent CTAs in two phases: ring steps t < split = ceil(N/2) (all N steps
+ * for N <= 2) as one unit per (step, pair of query tiles), step-major, starting
+ * on the rank's own block; then one unit per pair over steps [split, N), its
+ * online-softmax state kept on chip across them. Part t < split holds step t's
+ * partial, part split the merged partial of the remaining steps:
+ * cp_attn_ring_num_parts(plan) parts in all. Meanwhile two copy warps of every CTA fetch the blocks of
  * ranks rank+1, rank+2, ... (mod N), in that order, in 32 KiB chunks, from
  * pull_k[j] / pull_v[j] into slot j of k_all / v_all, counting finished chunks in
  * arrived[j]; a unit reads slot j once all of its chunks have arrived. The
@@ -215,10 +219,12 @@ CP_API int cp_attn_fwd_ring_step(cp_attn_plan_t plan, int rank, int step, const 
  *                  not NULL, a unit waits until arrived[j] >= 1, written by the
  *                  caller from outside this GPU's SMs (not by a copy that needs
  *                  them: the persistent kernel holds every SM)
- *   o_parts      : float32 [N][B*(S/N)*H][D], part t = step t, device (written)
- *   lse_parts    : float32 [N][B*(S/N)*H], device (written)
- * Rows as in cp_attn_fwd_ring_step; cp_merge_partials over the N parts gives the
+ *   o_parts      : float32 [P][B*(S/N)*H][D], P = cp_attn_ring_num_parts(plan),
+ *                  device (written)
+ *   lse_parts    : float32 [P][B*(S/N)*H], device (written)
+ * Rows as in cp_attn_fwd_ring_step; cp_merge_partials over the P parts gives the
  * rank's rows of full attention. Errors: as cp_attn_fwd_ring_step;
+ * CP_ERR_UNSUPPORTED for N > 255;
  * CP_ERR_INVALID_ARG for a missing pull source or arrived when pulling;
  * CP_ERR_UNSUPPORTED when pulling with N > 64; CP_ERR_ALIGNMENT for a pull
  * source not 16-byte or arrived not 4-byte aligned. A wait that runs out (2 s)
@@ -227,6 +233,10 @@ CP_API int cp_attn_fwd_ring_step(cp_attn_plan_t plan, int rank, int step, const 
 CP_API int cp_attn_fwd_ring(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all,
                             const void* const* pull_k, const void* const* pull_v, int* arrived,
                             float* o_parts, float* lse_parts, cp_stream_t stream);
+
+/* Number of partials cp_attn_fwd_ring writes (N for N <= 3, else ceil(N/2) + 1),
+ * or a negative status (CP_ERR_UNSUPPORTED for Ulysses). */
+CP_API int cp_attn_ring_num_parts(cp_attn_plan_t plan);
 
 /* Builds (and, with a device, uploads) the per-step schedules of one rank's ring
  * steps and of its one-launch forward. Idempotent. Errors: CP_ERR_INVALID_ARG, CP_ERR_UNSUPPORTED (Ulysses),
@@ -240,8 +250,9 @@ CP_API int cp_attn_ring_prepare(cp_attn_plan_t plan, int rank);
  * rank*B + b, head, query-tile pair, executed key tiles of the step, CTA) in
  * run order; when cta_loads is not NULL writes each CTA's modelled load (as
  * cp_attn_plan_cta_loads counts it; min(n, SM count) CTAs). step = -1 gives
- * the units of cp_attn_fwd_ring (N*B*H*pairs of them) with the query-tile pair
- * field holding pair | (ring step << 16).
+ * the units of cp_attn_fwd_ring with the query-tile pair field holding
+ * pair | (first step << 16) | (end step << 24) and the key-tile field the
+ * unit's total over its steps.
  */
 CP_API int64_t cp_attn_ring_schedule(cp_attn_plan_t plan, int rank, int step, int32_t* items,
                                      int64_t* cta_loads);

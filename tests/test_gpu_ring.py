@@ -70,11 +70,18 @@ def test_ring_step_matches_oracle_partials(B, H, S, D, N, layout, causal):
     (1, 2, 1024, 128, 4, "zigzag", True),
     (2, 2, 1536, 64, 3, "contiguous", True),
     (1, 3, 1920, 128, 5, "zigzag", True),
+    (1, 2, 4096, 128, 8, "zigzag", True),
+    (1, 2, 512, 64, 2, "contiguous", False),
 ])
 def test_ring_launch_equals_step_launches(B, H, S, D, N, layout, causal):
     q, k, v = make_small(B, H, S, D, 80 + N)
     plan = cp.Plan(B, H, S, D, N, causal, layout)
     qd, kd, vd = (G.to_layout(x, N, layout).cuda() for x in (q, k, v))
+    split = N if N <= 2 else (N + 1) // 2
+    assert plan.ring_parts() == (split + 1 if split < N else N)
+    f = lambda t: t.float().numpy()
+    parts = A.ring_partials(f(q), f(k), f(v), L.rank_major_map(B, S, N, layout), N, causal=causal)
+    T = S // N
     arrived = torch.zeros(N, dtype=torch.int32, device="cuda")
     for r in range(N):
         op, lp = cp.attn_fwd_ring(plan, r, qd[r], kd, vd)                  # every block resident
@@ -92,13 +99,24 @@ def test_ring_launch_equals_step_launches(B, H, S, D, N, layout, causal):
         if N > 1:
             chunks = -(-kd[0].numel() * 2 // 32768)
             assert arrived.tolist() == [0 if j == r else 2 * chunks for j in range(N)]
-        for t in range(N):
+        assert torch.equal(op.view(torch.int32), op2.view(torch.int32))
+        assert torch.equal(lp.view(torch.int32), lp2.view(torch.int32))
+        for t in range(split):               # first phase: the per-step partials, bit for bit
             rk = (r + t) % N
             os_, ls_ = cp.attn_fwd_ring_step(plan, r, t, qd[r], kd[rk].contiguous(), vd[rk].contiguous())
             assert torch.equal(op[t].view(torch.int32), os_.view(torch.int32)), (r, t)
             assert torch.equal(lp[t].view(torch.int32), ls_.view(torch.int32)), (r, t)
-        assert torch.equal(op.view(torch.int32), op2.view(torch.int32))
-        assert torch.equal(lp.view(torch.int32), lp2.view(torch.int32))
+        if split < N:                        # tail: the merge of steps split..N-1 (oracle)
+            o_ref, l_ref = A.merge([(parts[r][t][0].reshape(-1, D),
+                                     parts[r][t][1].transpose(0, 2, 1).reshape(-1)) for t in range(split, N)])
+            o_t = op[split].double().cpu().numpy()
+            l_t = lp[split].double().cpu().numpy()
+            fin = np.isfinite(l_ref)
+            assert np.array_equal(np.isfinite(l_t), fin)
+            d = np.abs(o_t - o_ref)
+            assert d.max() <= G.TOL_O_MAX and d.mean() <= G.TOL_O_MEAN, (r, d.max())
+            if fin.any():
+                assert np.abs(l_t[fin] - l_ref[fin]).max() <= G.TOL_LSE
     assert cp.check(plan) == 0
 
 
@@ -115,8 +133,8 @@ def test_ring_launch_times_out_on_a_block_that_never_arrives():
     arrived.fill_(1)
     op, lp = cp.attn_fwd_ring(plan, 0, qd[0], kd, vd, arrived=arrived)
     assert cp.check(plan) == 0
-    os_, ls_ = cp.attn_fwd_ring_step(plan, 0, 2, qd[0], kd[2].contiguous(), vd[2].contiguous())
-    assert torch.equal(op[2].view(torch.int32), os_.view(torch.int32))
+    os_, ls_ = cp.attn_fwd_ring_step(plan, 0, 1, qd[0], kd[1].contiguous(), vd[1].contiguous())
+    assert torch.equal(op[1].view(torch.int32), os_.view(torch.int32))
 
 
 def _run_ring(plan, qs, ks, vs, reps=1):

@@ -111,20 +111,26 @@ def test_ring_schedule_balance_zigzag_32k():
 def test_ring_launch_units_cover_every_step_once(S, N, layout, causal, B, H):
     p = cp.Plan(B, H, S, 128, N, causal, layout)
     npairs = -(-(S // N) // 256)
+    split = N if N <= 2 else (N + 1) // 2
+    assert p.ring_parts() == (split + 1 if split < N else N)
     for r in range(N):
         units, loads = p.ring_schedule(r, -1)
-        assert len(units) == N * B * H * npairs
-        seen = {(qp >> 16, rb, h, qp & 0xffff) for rb, h, qp, _, _ in units}
-        assert seen == {(t, r * B + b, h, qp) for t in range(N) for b in range(B) for h in range(H)
-                        for qp in range(npairs)}
-        walks = {t: _step_walk_lengths(S, N, layout, causal, r, t) for t in range(N)}
+        ranges = {}
         for rb, h, qp, cost, cta in units:
-            assert cost == walks[qp >> 16][qp & 0xffff]
-        # each CTA's units run in step order; CTAs are contiguous runs
+            t0, t1 = (qp >> 16) & 0xff, (qp >> 24) & 0xff
+            ranges.setdefault((rb, h, qp & 0xffff), []).append((t0, t1))
+            walks = [_step_walk_lengths(S, N, layout, causal, r, t)[qp & 0xffff] for t in range(t0, t1)]
+            assert cost == sum(walks)
+            # the first phase is one step per unit, the tail the remaining steps
+            assert (t1 == t0 + 1 and t0 < split) or (t0 == split and t1 == N)
+        assert set(ranges) == {(r * B + b, h, qp) for b in range(B) for h in range(H) for qp in range(npairs)}
+        for rs in ranges.values():          # every step of every pair exactly once
+            assert sorted(t for a, b in rs for t in range(a, b)) == list(range(N))
+        # each CTA's units run phase by phase; CTAs are contiguous runs
         assert [u[4] for u in units] == sorted(u[4] for u in units)
         for c in set(u[4] for u in units):
-            steps = [u[2] >> 16 for u in units if u[4] == c]
-            assert steps == sorted(steps)
+            phases = [(u[2] >> 16) & 0xff for u in units if u[4] == c]
+            assert phases == sorted(phases)
         assert sum(loads) == sum(2 * u[3] + 3 for u in units)
         assert max(loads) <= np.mean(loads) + max(2 * u[3] + 3 for u in units)
 
@@ -139,7 +145,8 @@ def test_ring_argument_validation():
     assert L.cp_attn_ring_prepare(p.handle, 3) == 0           # host schedules only without a device
     assert L.cp_attn_ring_schedule(p.handle, 0, 4, None, None) == -1
     assert L.cp_attn_ring_schedule(p.handle, 0, -2, None, None) == -1
-    assert L.cp_attn_ring_schedule(p.handle, 2, -1, None, None) == 4 * 2   # all steps' units
+    assert L.cp_attn_ring_schedule(p.handle, 2, -1, None, None) == 3 * 2   # steps 0, 1 and the tail [2, 4)
+    assert L.cp_attn_ring_num_parts(p.handle) == 3
     srcs = ctypes.cast((ctypes.c_void_p * 4)(16, 32, 48, 64), ctypes.c_void_p)
     bad_src = ctypes.cast((ctypes.c_void_p * 4)(16, 40, 48, 64), ctypes.c_void_p)
     null_src = ctypes.cast((ctypes.c_void_p * 4)(16, None, 48, 64), ctypes.c_void_p)
