@@ -183,7 +183,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["attn", "merge", "permute", "bwd"], default=None,
+    ap.add_argument("--profile", choices=["attn", "merge", "permute", "bwd", "ring"], default=None,
                     help="only launch one kernel warmup+steps times (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -245,8 +245,18 @@ def main():
             cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=lse)
             gq, gk, gv = (torch.empty_like(qz) for _ in range(3))
             bws = torch.empty(plan.bwd_workspace_bytes(), dtype=torch.uint8, device=dev)
+        if args.profile == "ring":
+            # rank 0's one-launch ring forward, fetching the other ranks' blocks
+            # (layout tensors standing in for their memory) into its own slots
+            rslots_k, rslots_v = torch.empty_like(kz), torch.empty_like(vz)
+            rslots_k[0].copy_(kz[0])
+            rslots_v[0].copy_(vz[0])
+            r_arr = torch.zeros(N, dtype=torch.int32, device=dev)
+            r_src = ([kz[j].data_ptr() for j in range(N)], [vz[j].data_ptr() for j in range(N)])
         for _ in range(args.warmup + args.steps):
-            if args.profile == "bwd":
+            if args.profile == "ring":
+                cp.attn_fwd_ring(plan, 0, qz[0], rslots_k, rslots_v, r_src[0], r_src[1], r_arr)
+            elif args.profile == "bwd":
                 cp.attn_bwd(plan, qz, kz, vz, oz, lse, dod, gq, gk, gv, bws)
             elif args.profile == "attn":
                 cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=lse)
