@@ -226,3 +226,37 @@ def test_ring_step_rejects_bad_arguments():
     with pytest.raises(cp.CpAttnError) as e:
         cp.attn_fwd_ring_step(plan, 0, 0, x.view(-1)[1:], x, x)      # 2 bytes past a 16-byte boundary
     assert e.value.status == -3
+
+
+@pytest.mark.parametrize("name,layout,rank", [("zigzag_32k", "zigzag", 3), ("long_128k", "contiguous", 2),
+                                              ("long_128k", "zigzag", 1)])
+def test_ring_rank_full_size_sampled_rows(name, layout, rank):
+    """One rank of a full-size workload, as bench.py runs it: one cooperative
+    launch fetching the other ranks' blocks, then the merge; the rank's rows among
+    the workload's sampled rows against the oracle."""
+    from workloads import sample_rows
+    w = WORKLOADS[name]
+    q, k, v = make_qkv(w)
+    N, T = w.N, w.S // w.N
+    plan = cp.Plan(w.B, w.H, w.S, w.D, N, w.causal, layout)
+    qd, kd, vd = (G.to_layout(x, N, layout).cuda() for x in (q, k, v))
+    ks, vs = torch.empty_like(kd), torch.empty_like(vd)
+    ks[rank].copy_(kd[rank])
+    vs[rank].copy_(vd[rank])
+    arrived = torch.zeros(N, dtype=torch.int32, device="cuda")
+    op, lp = cp.attn_fwd_ring(plan, rank, qd[rank], ks, vs, [kd[j].data_ptr() for j in range(N)],
+                              [vd[j].data_ptr() for j in range(N)], arrived)
+    o, lse = cp.merge_partials(op, lp)
+    assert cp.check(plan) == 0
+    del ks, vs, op, lp
+    pos = L.chunk_positions(w.S, N, layout)[rank]
+    local = {int(p): i for i, p in enumerate(pos)}
+    rows = np.array([r for r in sample_rows(w) if int(r[2]) in local])[:256]
+    assert len(rows) > 16
+    o_ref, l_ref = G.oracle_rows(q, k, v, rows, w.causal)
+    ix = torch.from_numpy(np.array([(r[0] * T + local[int(r[2])]) * w.H + r[1] for r in rows])).cuda()
+    got = o[ix].double().cpu().numpy()
+    got_l = lse[ix].double().cpu().numpy()
+    d = np.abs(got - o_ref)
+    assert d.max() <= G.TOL_O_MAX and d.mean() <= G.TOL_O_MEAN, d.max()
+    assert np.abs(got_l - l_ref).max() <= G.TOL_LSE
