@@ -1,16 +1,14 @@
 // ring.cu — host-side plumbing of the multi-GPU ring: device buffers that other
-// ranks' processes can map (CUDA IPC), and the transfer of a peer's key/value
-// block into this GPU's memory.
+// ranks' processes can map (CUDA IPC), and a device-to-device copy.
 //
 // Page "序列与上下文并行", section "上下文并行：注意力本身切分": every rank keeps
-// its own Q chunk and receives the K/V blocks of the other ranks one ring step at
-// a time, computing on the block it holds while the next one arrives; each step
-// moves one rank's K/V. On B200 the block is pulled from the peer's HBM by the
-// copy engine (a cudaMemcpyAsync between device pointers over NVLink), so the
-// transfer takes no SM away from the persistent attention kernel it overlaps,
-// and the attention kernel reads its keys and values from local memory only.
-// Ordering between ranks is left to the caller (host-side events and barriers);
-// nothing here waits on another GPU.
+// its own Q chunk and receives the K/V blocks of the other ranks, computing on
+// the blocks it holds while the next ones arrive. Each rank exposes its own block
+// in a slot buffer allocated here; the other ranks map it through CUDA IPC and
+// the copy warps of their one-launch ring forward read it over NVLink into local
+// slots (attn_fwd.cu). cp_copy_async is a plain cudaMemcpyAsync (the driver's own
+// fill of the local slot, and the per-step primitive's callers); such a copy can
+// need SM time, so no kernel waits for one. Nothing here waits on another GPU.
 #include <cuda_runtime.h>
 
 #include <cstdint>

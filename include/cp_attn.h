@@ -258,15 +258,17 @@ CP_API int64_t cp_attn_ring_schedule(cp_attn_plan_t plan, int rank, int step, in
                                      int64_t* cta_loads);
 
 /*
- * Plumbing of the multi-GPU ring (one process per GPU). A rank's receive slots
- * are allocated with cp_ring_buffer_alloc so that the neighbour's process can
- * map them: cp_ipc_get_handle writes the allocation's handle
- * (cp_ipc_handle_bytes() bytes, host memory) for the other process to pass to
- * cp_ipc_open_handle, which returns a device pointer to the peer's memory,
- * valid in this process until cp_ipc_close_handle. cp_copy_async enqueues one
- * copy of `bytes` between device pointers, a peer's included (copy engine,
- * over NVLink between GPUs); it does not wait for the peer, so the caller
- * orders it against the peer's writes and reads (host barrier plus events).
+ * Plumbing of the multi-GPU ring (one process per GPU). A rank's slot buffer is
+ * allocated with cp_ring_buffer_alloc so that the other ranks' processes can map
+ * it: cp_ipc_get_handle writes the allocation's handle (cp_ipc_handle_bytes()
+ * bytes, host memory) for another process to pass to cp_ipc_open_handle, which
+ * returns a device pointer to the peer's memory, valid in this process until
+ * cp_ipc_close_handle (the pointer cp_attn_fwd_ring's copy warps read from).
+ * cp_copy_async enqueues one cudaMemcpyAsync of `bytes` between device pointers
+ * (a peer's included) on `stream`; it does not wait for the peer, so the caller
+ * orders it against the peer's writes and reads. Such a copy can need SM time:
+ * one issued on a side stream did not progress while a persistent kernel held
+ * every SM, so no kernel may wait for it.
  * Errors: CP_ERR_INVALID_ARG (null pointer, zero-byte allocation), CP_ERR_CUDA.
  */
 CP_API int cp_ring_buffer_alloc(size_t bytes, void** out);
