@@ -15,7 +15,7 @@ Sources on the pages:
   * Same page, section "工程实践" (practice): positions are global positions
     under context parallelism.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   * the causal mask keeps key j for query i iff pos(j) <= pos(i) (diagonal
     kept), in global positions;
   * lse is the natural logarithm of the sum of exp of the *scaled* scores;

@@ -8,7 +8,7 @@ without writing it out; their only printed position encoding is the sinusoidal
 one of page "Tensor并行与算子拆分" (aiknowledge.cn), the PositionalEncoding class
 of its model example: frequencies 10000^(-2i/d) on the even/odd feature pairs.
 
-Reading (stated in the design doc): rotary embedding with that base and pairing —
+Reading, where the pages name no rotary formula: rotary embedding with that base and pairing —
 feature pair (2i, 2i+1) of a head vector at global position p is rotated by the
 angle p * theta_i, theta_i = base^(-2i/D):
     y[2i]   = x[2i] cos(p theta_i) - x[2i+1] sin(p theta_i)

@@ -16,7 +16,7 @@ Sources on the pages:
     draw exceeds the drop rate, kept values divided by 1 - rate); its check that
     the per-shard results, concatenated, equal LayerNorm of the whole sequence.
 
-Readings (listed in the design doc): the fused op after a tensor-parallel region is
+Readings where the pages leave it open: the fused op after a tensor-parallel region is
     z = dropout(reduce_scatter(partials)) + residual,   y = LayerNorm(z),
 with the keep mask an input (the random draw the method makes); reduce-scatter
 over N ranks sums the N partial [S, ...] tensors and hands rank i its i-th
