@@ -51,6 +51,7 @@ SIGNATURES = {
     "cp_attn_ring_prepare": (_I, [_P, _I]),
     "cp_attn_ring_num_parts": (_I, [_P]),
     "cp_attn_fwd_ring": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "cp_attn_fwd_ring_external": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P]),
     "cp_attn_ring_schedule": (_I64, [_P, _I, _I, _P, _P]),
     "cp_ring_buffer_alloc": (_I, [_SZ, ctypes.POINTER(_P)]),
     "cp_ring_buffer_free": (_I, [_P]),
@@ -269,6 +270,23 @@ def attn_fwd_ring(plan: Plan, rank: int, q, k_all, v_all, pull_k=None, pull_v=No
     return o_parts, lse_parts
 
 
+def attn_fwd_ring_external(plan: Plan, rank: int, q, k_all, v_all, arrived, o_parts=None, lse_parts=None,
+                           stream=None):
+    """``cp_attn_fwd_ring_external``: as ``attn_fwd_ring`` without pull sources,
+    each unit waiting (bounded) until ``arrived[j] >= 1`` before it reads slot j;
+    the caller's own transfer fills the slots and raises the counts."""
+    rows = plan.B * (plan.S // plan.N) * plan.H
+    P = plan.ring_parts()
+    if o_parts is None:
+        o_parts = torch.empty(P, rows, plan.D, dtype=torch.float32, device=q.device)
+    if lse_parts is None:
+        lse_parts = torch.empty(P, rows, dtype=torch.float32, device=q.device)
+    _check("cp_attn_fwd_ring_external",
+           lib().cp_attn_fwd_ring_external(plan.handle, int(rank), _ptr(q), _vp_of(k_all), _vp_of(v_all),
+                                           _vp_of(arrived), _ptr(o_parts), _ptr(lse_parts), _stream(stream)))
+    return o_parts, lse_parts
+
+
 def _vp_of(x):
     return ctypes.c_void_p(int(x) if isinstance(x, int) else x.data_ptr())
 
@@ -441,6 +459,18 @@ def attn_fwd_ulysses_noalloc(plan: Plan, q, k, v, o, lse=None, stream=None):
     workspace, so ``o`` (and ``lse`` if wanted) must be passed in. Calls that
     may overlap on the GPU share that scratch and must be serialised.
     """
+    if plan.layout != "ulysses":
+        raise ValueError("attn_fwd_ulysses_noalloc needs a Ulysses plan")
+    B, H, S, D, N = plan.B, plan.H, plan.S, plan.D, plan.N
+    shape = (N, B, S // N, H, D)
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != shape or not t.is_contiguous() or t.device.type != "cuda":
+            raise ValueError(f"{name}: expected a contiguous bf16 CUDA tensor of shape {shape}")
+    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, S) or not lse.is_contiguous()
+                            or lse.device != o.device):
+        raise ValueError(f"lse: expected a contiguous float32 tensor of shape {(B, H, S)} on {o.device}")
+    if any(t.device != o.device for t in (q, k, v)):
+        raise ValueError("q, k, v and o must be on one device")
     _check("cp_attn_fwd_ulysses_noalloc",
            lib().cp_attn_fwd_ulysses_noalloc(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                                             _stream(stream)))

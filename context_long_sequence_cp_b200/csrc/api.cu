@@ -853,9 +853,17 @@ int cp_attn_fwd_ring_step(cp_attn_plan_t plan, int rank, int step, const void* q
   return launch_attn_fwd(L, plan->D, true, static_cast<cudaStream_t>(stream)) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
 
-int cp_attn_fwd_ring(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all,
-                     const void* const* pull_k, const void* const* pull_v, int* arrived, float* o_parts,
-                     float* lse_parts, cp_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// One rank's whole ring forward in one launch. Three arrival modes: pulling (the
+// kernel's copy warps fetch the other blocks and count their chunks in arrived),
+// external (arrived[j] >= 1 is set by the caller's own transfer) and resident
+// (arrived NULL: every slot already holds its block, no wait).
+int ring_launch(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all, const void* const* pull_k,
+                const void* const* pull_v, int* arrived, bool external, float* o_parts, float* lse_parts,
+                cp_stream_t stream) {
   if (plan == nullptr || q == nullptr || k_all == nullptr || v_all == nullptr || o_parts == nullptr ||
       lse_parts == nullptr)
     return CP_ERR_INVALID_ARG;
@@ -864,6 +872,11 @@ int cp_attn_fwd_ring(cp_attn_plan_t plan, int rank, const void* q, void* k_all, 
   if ((pull_k == nullptr) != (pull_v == nullptr)) return CP_ERR_INVALID_ARG;
   const bool pull = pull_k != nullptr && plan->N > 1;
   if (pull && arrived == nullptr) return CP_ERR_INVALID_ARG;
+  // Without pull sources a wait on arrived counts is only made on request: a
+  // stale arrived buffer passed by mistake would otherwise stall every unit
+  // until its wait runs out.
+  if (!pull && !external && arrived != nullptr) return CP_ERR_INVALID_ARG;
+  if (external && arrived == nullptr) return CP_ERR_INVALID_ARG;
   if (pull && plan->N > kMaxPullRanks) return CP_ERR_UNSUPPORTED;
   if (plan->N > 255) return CP_ERR_UNSUPPORTED;   // unit steps are packed in 8 bits
   if (!aligned16(q) || !aligned16(k_all) || !aligned16(v_all) || !aligned16(o_parts) || !aligned16(lse_parts) ||
@@ -923,6 +936,21 @@ int cp_attn_fwd_ring(cp_attn_plan_t plan, int rank, const void* q, void* k_all, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (pull && cudaMemsetAsync(arrived, 0, sizeof(int) * plan->N, st) != cudaSuccess) return CP_ERR_CUDA;
   return launch_attn_fwd(L, plan->D, true, st) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int cp_attn_fwd_ring(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all,
+                     const void* const* pull_k, const void* const* pull_v, int* arrived, float* o_parts,
+                     float* lse_parts, cp_stream_t stream) {
+  return ring_launch(plan, rank, q, k_all, v_all, pull_k, pull_v, arrived, false, o_parts, lse_parts, stream);
+}
+
+int cp_attn_fwd_ring_external(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all,
+                              int* arrived, float* o_parts, float* lse_parts, cp_stream_t stream) {
+  return ring_launch(plan, rank, q, k_all, v_all, nullptr, nullptr, arrived, true, o_parts, lse_parts, stream);
 }
 
 int cp_merge_partials(int num_parts, int64_t rows, int D, const float* o_parts, const float* lse_parts,
@@ -1059,6 +1087,9 @@ int cp_debug_wait_timeout_probe(cp_attn_plan_t plan, int timeout_us, cp_stream_t
 }
 
 }  // extern "C"
+
+// The device a plan was made on (-1 without a device).
+int cp_internal_plan_device(const cp_attn_plan_s* plan) { return plan == nullptr ? -1 : plan->device; }
 
 // Ulysses forward on a caller-chosen scratch buffer: the same launches as the
 // Ulysses branch of cp_attn_fwd, with the head-group copies placed in `scratch`.

@@ -71,12 +71,12 @@ struct FwdLaunch {
 cudaError_t launch_attn_fwd(const FwdLaunch& L, int D, bool partial, cudaStream_t stream);
 size_t attn_fwd_smem_bytes(int D);
 
-// merge.cu
+// merge_permute.cu: merge of partials
 cudaError_t launch_merge(int num_parts, int64_t rows, int D, const float* o_parts,
                          const float* lse_parts, __nv_bfloat16* o_out, float* lse_out,
                          cudaStream_t stream);
 
-// permute.cu
+// merge_permute.cu: layout maps
 struct PermuteArgs {
   int kind;          // 0: contiguous/zigzag token rows; 1: Ulysses head-group runs
   int direction;     // 0: forward gather, 1: inverse
@@ -96,7 +96,7 @@ struct RopeArgs {
 cudaError_t launch_rope_permute(const PermuteArgs& a, const RopeArgs& ra, const void* in, void* out,
                                 cudaStream_t stream);
 
-// probe.cu
+// merge_permute.cu: the bounded-wait self-test (a wait on a barrier nothing arrives on)
 cudaError_t launch_wait_probe(int* status, uint64_t limit_ns, cudaStream_t stream);
 
 }  // namespace cpattn
@@ -104,10 +104,7 @@ cudaError_t launch_wait_probe(int* status, uint64_t limit_ns, cudaStream_t strea
 // api.cu: the Ulysses forward with a caller-chosen scratch buffer of at least
 // cp_attn_workspace_bytes(plan, 0) bytes (used by the no-alloc entry point).
 struct cp_attn_plan_s;
+int cp_internal_plan_device(const cp_attn_plan_s* plan);
 int cp_internal_ulysses_fwd_scratch(cp_attn_plan_s* plan, const void* q, const void* k, const void* v,
                                     void* o, float* lse, void* scratch, size_t scratch_bytes,
                                     cudaStream_t stream);
-
-namespace cpattn {
-
-}  // namespace cpattn

@@ -28,9 +28,12 @@ std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device (first call: look it up).
-int scratch_on_current_device(void** out) {
+// The current device must be the plan's: the plan's work list and status word
+// live there, and a kernel given another GPU's scratch would read the wrong memory.
+int scratch_on_current_device(int plan_device, void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CP_ERR_CUDA;
+  if (dev != plan_device) return CP_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
@@ -51,7 +54,7 @@ extern "C" CP_API int cp_attn_fwd_ulysses_noalloc(cp_attn_plan_t plan, const voi
   if (need == 0) return CP_ERR_UNSUPPORTED;                       // not a Ulysses plan
   if (need > CP_NOALLOC_SCRATCH_BYTES) return CP_ERR_WORKSPACE;   // beyond the fixed scratch
   void* scratch = nullptr;
-  const int rc = scratch_on_current_device(&scratch);
+  const int rc = scratch_on_current_device(cp_internal_plan_device(plan), &scratch);
   if (rc != CP_OK) return rc;
   return cp_internal_ulysses_fwd_scratch(plan, q, k, v, o, lse, scratch, CP_NOALLOC_SCRATCH_BYTES,
                                          static_cast<cudaStream_t>(stream));

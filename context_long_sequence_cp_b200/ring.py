@@ -140,7 +140,8 @@ class RingRank:
         def launch():
             st.wait_event(self.fill_done)
             pk, pv = self.pull_sources(c) if N > 1 else (None, None)
-            _launch_ring(self.plan, r, q, k_all, v_all, pk, pv, self.arrived, self.o_parts, self.lse_parts, st)
+            _launch_ring(self.plan, r, q, k_all, v_all, pk, pv, self.arrived if N > 1 else None, self.o_parts,
+                         self.lse_parts, st)
 
         run_ring(fill, self.fill_done.synchronize, self.barrier, launch)
         o, lse = merge_partials(self.o_parts, self.lse_parts, stream=st)
@@ -158,7 +159,8 @@ def _launch_ring(plan, rank, q, k_all, v_all, pk, pv, arrived, o_parts, lse_part
         pva = ctypes.cast((ctypes.c_void_p * len(pv))(*pv), ctypes.c_void_p)
     _check("cp_attn_fwd_ring",
            lib().cp_attn_fwd_ring(plan.handle, rank, _vp(q.data_ptr()), _vp(k_all), _vp(v_all), pka, pva,
-                                  _vp(arrived.data_ptr()), _vp(o_parts.data_ptr()), _vp(lse_parts.data_ptr()),
+                                  None if arrived is None else _vp(arrived.data_ptr()), _vp(o_parts.data_ptr()),
+                                  _vp(lse_parts.data_ptr()),
                                   _vp(st.cuda_stream)))
 
 

@@ -214,18 +214,18 @@ CP_API int cp_attn_fwd_ring_step(cp_attn_plan_t plan, int rank, int step, const 
  *                  K/V block [B][S/N][H][D] as addressable from this GPU (entry
  *                  `rank` unused), 16-byte aligned, unchanged until the kernel
  *                  ends; both NULL: no pull, every slot already holds its block
- *   arrived      : int32 [N] device workspace (set to 0 on `stream` before the
- *                  launch when pulling). Without pull sources and with arrived
- *                  not NULL, a unit waits until arrived[j] >= 1, written by the
- *                  caller from outside this GPU's SMs (not by a copy that needs
- *                  them: the persistent kernel holds every SM)
+ *   arrived      : int32 [N] device workspace, needed when pulling (set to 0
+ *                  on `stream` before the launch); must be NULL without pull
+ *                  sources (see cp_attn_fwd_ring_external for a wait on
+ *                  arrivals the caller raises)
  *   o_parts      : float32 [P][B*(S/N)*H][D], P = cp_attn_ring_num_parts(plan),
  *                  device (written)
  *   lse_parts    : float32 [P][B*(S/N)*H], device (written)
  * Rows as in cp_attn_fwd_ring_step; cp_merge_partials over the P parts gives the
  * rank's rows of full attention. Errors: as cp_attn_fwd_ring_step;
  * CP_ERR_UNSUPPORTED for N > 255;
- * CP_ERR_INVALID_ARG for a missing pull source or arrived when pulling;
+ * CP_ERR_INVALID_ARG for a missing pull source or arrived when pulling, and
+ * for a non-NULL arrived without pull sources;
  * CP_ERR_UNSUPPORTED when pulling with N > 64; CP_ERR_ALIGNMENT for a pull
  * source not 16-byte or arrived not 4-byte aligned. A wait that runs out (2 s)
  * ends the kernel with CP_ERR_TIMEOUT in cp_attn_check.
@@ -233,6 +233,21 @@ CP_API int cp_attn_fwd_ring_step(cp_attn_plan_t plan, int rank, int step, const 
 CP_API int cp_attn_fwd_ring(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all,
                             const void* const* pull_k, const void* const* pull_v, int* arrived,
                             float* o_parts, float* lse_parts, cp_stream_t stream);
+
+/* cp_attn_fwd_ring without pull sources, for a caller whose own transfer fills
+ * the other ranks' slots while the launch runs: before its first read of slot
+ * j != rank a unit waits until arrived[j] >= 1 (slot j complete, stores visible
+ * at GPU scope), then reads it. The caller raises arrived[j] from outside this
+ * GPU's SMs (a peer's stores, the host through mapped memory), not by a copy
+ * that needs them: the persistent kernel holds every SM. arrived is not reset
+ * here. Same page and section as cp_attn_fwd_ring; same arguments without
+ * pull_k / pull_v.
+ *   arrived : int32 [N] device, 4-byte aligned, required (CP_ERR_INVALID_ARG
+ *             when NULL)
+ * A wait that runs out (2 s) ends the kernel with CP_ERR_TIMEOUT in
+ * cp_attn_check; the context stays usable. */
+CP_API int cp_attn_fwd_ring_external(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all,
+                                     int* arrived, float* o_parts, float* lse_parts, cp_stream_t stream);
 
 /* Number of partials cp_attn_fwd_ring writes (N for N <= 3, else ceil(N/2) + 1),
  * or a negative status (CP_ERR_UNSUPPORTED for Ulysses). */
@@ -469,6 +484,10 @@ CP_API int cp_debug_wait_timeout_probe(cp_attn_plan_t plan, int timeout_us, cp_s
  *     byte it reads. Two calls whose work can overlap on the GPU (different
  *     streams without ordering, or different host threads) race on it:
  *     serialise them.
+ *   - The current device must be the one the plan was made on, and `stream`
+ *     must belong to it: the scratch used is the current device's, the work
+ *     list and status word are the plan's. A call made with another device
+ *     current returns CP_ERR_INVALID_ARG and launches nothing.
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
  */
 #define CP_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)

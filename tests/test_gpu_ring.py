@@ -125,13 +125,13 @@ def test_ring_launch_times_out_on_a_block_that_never_arrives():
     q, k, v = make_small(B, H, S, D, 90)
     plan = cp.Plan(B, H, S, D, N, True, "zigzag")
     qd, kd, vd = (G.to_layout(x, N, "zigzag").cuda() for x in (q, k, v))
-    arrived = torch.zeros(N, dtype=torch.int32, device="cuda")     # no pull, nothing raises the counts
-    cp.attn_fwd_ring(plan, 0, qd[0], kd, vd, arrived=arrived)
+    arrived = torch.zeros(N, dtype=torch.int32, device="cuda")     # nothing raises the counts
+    cp.attn_fwd_ring_external(plan, 0, qd[0], kd, vd, arrived)
     assert cp.check(plan) == -5                                    # CP_ERR_TIMEOUT, after the 2 s budget
     assert cp.check(plan) == 0
     # the context is still usable: the same launch with the blocks marked arrived
     arrived.fill_(1)
-    op, lp = cp.attn_fwd_ring(plan, 0, qd[0], kd, vd, arrived=arrived)
+    op, lp = cp.attn_fwd_ring_external(plan, 0, qd[0], kd, vd, arrived)
     assert cp.check(plan) == 0
     os_, ls_ = cp.attn_fwd_ring_step(plan, 0, 1, qd[0], kd[1].contiguous(), vd[1].contiguous())
     assert torch.equal(op[1].view(torch.int32), os_.view(torch.int32))

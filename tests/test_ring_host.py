@@ -157,7 +157,14 @@ def test_ring_argument_validation():
     assert ring(0, buf, buf, buf, srcs, srcs, None, buf, buf, None) == -1         # pulling needs arrived
     assert ring(0, buf, buf, buf, null_src, srcs, buf, buf, buf, None) == -1      # a missing source
     assert ring(0, buf, buf, buf, bad_src, srcs, buf, buf, buf, None) == -3       # a misaligned source
-    assert ring(0, buf, buf, buf, None, None, ctypes.c_void_p(18), buf, buf, None) == -3
+    # without pull sources an arrived buffer is refused (a stale one would stall
+    # every unit until its wait runs out); the explicit external-arrival entry
+    # takes it, and refuses a missing or misaligned one
+    assert ring(0, buf, buf, buf, None, None, buf, buf, buf, None) == -1
+    ext = lambda *a: L.cp_attn_fwd_ring_external(p.handle, *a)
+    assert ext(0, buf, buf, buf, None, buf, buf, None) == -1
+    assert ext(0, buf, buf, buf, ctypes.c_void_p(18), buf, buf, None) == -3
+    assert ext(4, buf, buf, buf, buf, buf, buf, None) == -1
     big = cp.Plan(1, 2, 65 * 256, 64, 65, False, "contiguous")
     srcs65 = ctypes.cast((ctypes.c_void_p * 65)(*([16] * 65)), ctypes.c_void_p)
     assert L.cp_attn_fwd_ring(big.handle, 0, buf, buf, buf, srcs65, srcs65, buf, buf, buf, None) == -2
