@@ -10,7 +10,7 @@
 //   Dr = rowsum(dO * O),  dS = P * (dP - Dr),  dQ = scale dS K,  dK = scale dS^T Q.
 //
 // Three kernels, no atomics (results are deterministic):
-//   bwd_pre_kernel     per view row: lse2 = lse * log2(e) and Dr, stored
+//   bwd_pre_kernel     per view row: nlse2 = -lse * log2(e) and Dr, stored
 //                      [NR*B][Hh][T] so that a query tile's 128 values are
 //                      contiguous (one bulk copy).
 //   attn_bwd_kv_kernel one 128-key tile per work item; walks the query tiles
@@ -142,7 +142,8 @@ __device__ __forceinline__ void store_row_bf16(uint32_t tAcc, bool have, float m
 
 // ------------------------------------------------------------------ preprocess
 // One warp per view row: Dr = sum_d dO * O (fp32), and the row's lse in log2
-// units, both stored [NR*B][Hh][T].
+// units, negated (so that P = exp2(fma(s, scale_log2, nlse2))), both stored
+// [NR*B][Hh][T].
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdPreParams p) {
   const Geometry g = p.g;
@@ -150,6 +151,10 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdPreParams p) {
   const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int64_t rows = static_cast<int64_t>(g.NR) * g.B * g.T * g.Hh;
+  // The dK/dV kernel's 512-byte copies of a ragged last query tile read up to
+  // 127 values past the end of each array: zero dvec's padding, so that a masked
+  // column's P = 0 times (dP - Dr) stays 0 (lse2's over-read lands in dvec).
+  if (blockIdx.x == 0 && threadIdx.x < kTile) p.dvec[rows + threadIdx.x] = 0.f;
   constexpr int E = D / 32;   // elements per lane: 4 (D = 128) or 2 (D = 64)
   for (int64_t r = warp0; r < rows; r += nwarps) {
     const __nv_bfloat16* orow = p.o + r * D + lane * E;
@@ -182,7 +187,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdPreParams p) {
       const int64_t li = (static_cast<int64_t>(bv % p.lse_B) * p.lse_H + (bv / p.lse_B) * g.Hh + h) * p.lse_S + gq;
       const float l = __ldg(p.lse + li);
       const int64_t wi = (static_cast<int64_t>(rb) * g.Hh + h) * g.T + t;
-      p.lse2[wi] = l == -INFINITY ? INFINITY : l * kLog2e;
+      p.lse2[wi] = l == -INFINITY ? -INFINITY : -l * kLog2e;
       p.dvec[wi] = acc;
     }
   }
@@ -460,8 +465,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (g.causal) lo = clamp_int(static_cast<int64_t>(count_le(g, rq, kpos - 1)) - q0, 0, kTile);
           if (!valid_k) lo = hi;
         }
-        const float* l2 = sm.lse2[st];
+        const float* nl2 = sm.lse2[st];
         const float* dr = sm.dvec[st];
+        // Whole tiles take the packed path: no column limits, two columns per
+        // f32x2 instruction, the statistics read in pairs. The class is the same
+        // for every thread of the CTA (one walk entry per tile), so the branch
+        // is uniform; the TMEM stores below are outside it.
+        const bool whole = entry_c0(ent) == kFull;
         // P^T of this warpgroup's 64 query columns from S^T, packed to bf16 (the
         // values dV's product uses; dS^T below is formed from the same values).
         uint32_t pk[32];
@@ -470,15 +480,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld32x2(tA + wg * 64, tA + wg * 64 + 32, sa, sb);
           tc_fence_before();
           mbar_arrive(smem_addr(&sm.s_free));   // region A may take dP^T
+          if (whole) {
+            const uint64_t sl2_2 = f2_pack(sl2, sl2);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int c = wg * 64 + 2 * j;
-            const float p0 = (c >= lo && c < hi) ? ex2_approx(__uint_as_float(sa[2 * j]) * sl2 - l2[c]) : 0.f;
-            const float p1 = (c + 1 >= lo && c + 1 < hi) ? ex2_approx(__uint_as_float(sa[2 * j + 1]) * sl2 - l2[c + 1]) : 0.f;
-            const float p2 = (c + 32 >= lo && c + 32 < hi) ? ex2_approx(__uint_as_float(sb[2 * j]) * sl2 - l2[c + 32]) : 0.f;
-            const float p3 = (c + 33 >= lo && c + 33 < hi) ? ex2_approx(__uint_as_float(sb[2 * j + 1]) * sl2 - l2[c + 33]) : 0.f;
-            pk[j] = pack_bf16x2(p0, p1);
-            pk[16 + j] = pack_bf16x2(p2, p3);
+            for (int j = 0; j < 16; ++j) {
+              const int c = wg * 64 + 2 * j;
+              const uint64_t na = *reinterpret_cast<const uint64_t*>(nl2 + c);
+              const uint64_t nb = *reinterpret_cast<const uint64_t*>(nl2 + c + 32);
+              float x0, x1, x2, x3;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(sa[2 * j]), __uint_as_float(sa[2 * j + 1])), sl2_2, na), x0, x1);
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(sb[2 * j]), __uint_as_float(sb[2 * j + 1])), sl2_2, nb), x2, x3);
+              pk[j] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+              pk[16 + j] = pack_bf16x2(ex2_approx(x2), ex2_approx(x3));
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int c = wg * 64 + 2 * j;
+              const float p0 = (c >= lo && c < hi) ? ex2_approx(fmaf(__uint_as_float(sa[2 * j]), sl2, nl2[c])) : 0.f;
+              const float p1 =
+                  (c + 1 >= lo && c + 1 < hi) ? ex2_approx(fmaf(__uint_as_float(sa[2 * j + 1]), sl2, nl2[c + 1])) : 0.f;
+              const float p2 =
+                  (c + 32 >= lo && c + 32 < hi) ? ex2_approx(fmaf(__uint_as_float(sb[2 * j]), sl2, nl2[c + 32])) : 0.f;
+              const float p3 = (c + 33 >= lo && c + 33 < hi)
+                                   ? ex2_approx(fmaf(__uint_as_float(sb[2 * j + 1]), sl2, nl2[c + 33]))
+                                   : 0.f;
+              pk[j] = pack_bf16x2(p0, p1);
+              pk[16 + j] = pack_bf16x2(p2, p3);
+            }
           }
         }
         ok = mbar_wait(smem_addr(&sm.dp_full), d_cnt & 1, ctl);
@@ -492,13 +521,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld32x2(tA + wg * 64, tA + wg * 64 + 32, da, db);
           tc_fence_before();
           mbar_arrive(smem_addr(&sm.a_free));   // region A may take the next S^T
+          // dS^T = P^T * (dP^T - Dr), two columns per f32x2 instruction (masked
+          // columns have P = 0, so the same form serves every tile).
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int c = wg * 64 + 2 * j;
-            const float d0 = __uint_as_float(pk[j] << 16) * (__uint_as_float(da[2 * j]) - dr[c]);
-            const float d1 = __uint_as_float(pk[j] & 0xffff0000u) * (__uint_as_float(da[2 * j + 1]) - dr[c + 1]);
-            const float d2 = __uint_as_float(pk[16 + j] << 16) * (__uint_as_float(db[2 * j]) - dr[c + 32]);
-            const float d3 = __uint_as_float(pk[16 + j] & 0xffff0000u) * (__uint_as_float(db[2 * j + 1]) - dr[c + 33]);
+            const uint64_t ra = *reinterpret_cast<const uint64_t*>(dr + c);
+            const uint64_t rb = *reinterpret_cast<const uint64_t*>(dr + c + 32);
+            const uint64_t ga = f2_sub(f2_pack(__uint_as_float(da[2 * j]), __uint_as_float(da[2 * j + 1])), ra);
+            const uint64_t gb = f2_sub(f2_pack(__uint_as_float(db[2 * j]), __uint_as_float(db[2 * j + 1])), rb);
+            float d0, d1, d2, d3;
+            f2_unpack(f2_mul(bf16x2_to_f2(pk[j]), ga), d0, d1);
+            f2_unpack(f2_mul(bf16x2_to_f2(pk[16 + j]), gb), d2, d3);
             dk[j] = pack_bf16x2(d0, d1);
             dk[16 + j] = pack_bf16x2(d2, d3);
           }
@@ -732,7 +766,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool valid = tl < g.T;
       const int64_t gq = global_pos(g, rq, valid ? tl : g.T - 1);
       const int64_t vi = (static_cast<int64_t>(w.rb) * g.Hh + w.h) * g.T + (valid ? tl : 0);
-      const float lse2 = valid ? __ldg(p.lse2 + vi) : INFINITY;
+      const float nlse2 = valid ? __ldg(p.lse2 + vi) : -INFINITY;
       const float drow = valid ? __ldg(p.dvec + vi) : 0.f;
       const int* off = p.walk_off + rq * p.ntiles + w.qp;
       const int e_begin = __ldg(off), e_end = __ldg(off + 1);
@@ -757,22 +791,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_before();
         mbar_arrive(smem_addr(&sm.sdp_free));
         const uint32_t tbuf = tdS + (ntile & 1) * 64 + wg * 32;
+        // Whole tiles (the class is the same for every thread of the CTA, so the
+        // branch is uniform) take the packed path: two columns per f32x2
+        // instruction, no column limit. The TMEM stores are outside the branch.
+        const bool whole = entry_c0(ent) == kFull;
+        uint32_t dk[2][16];
+        if (whole) {
+          const uint64_t sl2_2 = f2_pack(sl2, sl2), nl_2 = f2_pack(nlse2, nlse2), dr_2 = f2_pack(drow, drow);
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int col0 = wg * 64 + cc * 32;
-          uint32_t dk[16];
+          for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int c = col0 + 2 * j;
-            const bool a0 = c < lim, a1 = c + 1 < lim;
-            const float p0 = a0 ? ex2_approx(__uint_as_float(sa[cc][2 * j]) * sl2 - lse2) : 0.f;
-            const float p1 = a1 ? ex2_approx(__uint_as_float(sa[cc][2 * j + 1]) * sl2 - lse2) : 0.f;
-            const float d0 = a0 ? p0 * (__uint_as_float(da[cc][2 * j]) - drow) : 0.f;
-            const float d1 = a1 ? p1 * (__uint_as_float(da[cc][2 * j + 1]) - drow) : 0.f;
-            dk[j] = pack_bf16x2(d0, d1);
+            for (int j = 0; j < 16; ++j) {
+              float x0, x1, d0, d1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(sa[cc][2 * j]), __uint_as_float(sa[cc][2 * j + 1])), sl2_2,
+                               nl_2),
+                        x0, x1);
+              const uint64_t g2 =
+                  f2_sub(f2_pack(__uint_as_float(da[cc][2 * j]), __uint_as_float(da[cc][2 * j + 1])), dr_2);
+              f2_unpack(f2_mul(f2_pack(ex2_approx(x0), ex2_approx(x1)), g2), d0, d1);
+              dk[cc][j] = pack_bf16x2(d0, d1);
+            }
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int col0 = wg * 64 + cc * 32;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int c = col0 + 2 * j;
+              const bool a0 = c < lim, a1 = c + 1 < lim;
+              const float p0 = a0 ? ex2_approx(fmaf(__uint_as_float(sa[cc][2 * j]), sl2, nlse2)) : 0.f;
+              const float p1 = a1 ? ex2_approx(fmaf(__uint_as_float(sa[cc][2 * j + 1]), sl2, nlse2)) : 0.f;
+              const float d0 = a0 ? p0 * (__uint_as_float(da[cc][2 * j]) - drow) : 0.f;
+              const float d1 = a1 ? p1 * (__uint_as_float(da[cc][2 * j + 1]) - drow) : 0.f;
+              dk[cc][j] = pack_bf16x2(d0, d1);
+            }
           }
-          tmem_st16(tbuf + cc * 16, dk);
         }
+        tmem_st16(tbuf, dk[0]);
+        tmem_st16(tbuf + 16, dk[1]);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(smem_addr(&sm.p_full[wg]));

@@ -12,8 +12,8 @@
 namespace cpattn {
 
 // Row statistics of the backward, per view row (rb, h, t) stored [NR*B][Hh][T]:
-// lse2 = lse * log2(e) (+inf where lse is -inf, so that exp2(s - lse2) is 0) and
-// dvec = rowsum(dO * O).
+// lse2 = -lse * log2(e), the negated lse in log2 units (-inf where lse is -inf,
+// so that exp2(s * scale_log2 + lse2) is 0), and dvec = rowsum(dO * O).
 struct BwdPreParams {
   Geometry g;
   const __nv_bfloat16* o;      // forward output, view layout [NR*B][T][Hh][D]
