@@ -22,9 +22,15 @@ instead and time each launch between its own events, the flush enqueued ahead
 so that no host latency falls inside a pair.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
-                       [--workload NAME]
-Under torchrun every rank runs its own replica of the workload (independent
-problems, no data-path collective: weak scaling) and rank 0 prints the line.
+                       [--workload NAME] [--mode ring|replica]
+Under torchrun (N > 1) the default mode is the context-parallel ring itself:
+rank r holds chunk r of the workload's sequence (its zigzag or contiguous
+share), the N ranks run the ring forward over CUDA IPC (``ring.IpcRing``: each
+rank fetches the other ranks' K/V blocks over NVLink inside its one-launch
+forward), and the line reports the whole problem's FLOPs over the slowest
+rank's time (strong scaling: the total work is fixed). ``--mode replica``
+instead runs an independent replica of the one-GPU problem per rank (weak
+scaling). Rank 0 prints the line.
 """
 from __future__ import annotations
 
@@ -520,6 +526,152 @@ def ring_components(cp, torch, plan, w, dev, stream, legs, qz, kz, vz, oz, att_m
     }
 
 
+# ----------------------------------------------------------------------------- ring mode (N > 1)
+
+def timed_ring_steps(step, barrier, events, steps: int, warmup: int) -> float:
+    """``warmup`` untimed steps, then ``steps`` steps between one pair of events,
+    bracketed by ``barrier()`` (host barrier of all ranks + device synchronise)
+    on both sides; returns this rank's milliseconds per step. ``events()``
+    returns a (start, end) pair with ``record()`` and ``elapsed_time(end)``."""
+    for _ in range(warmup):
+        step()
+    barrier()
+    e0, e1 = events()
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    barrier()
+    return e0.elapsed_time(e1) / steps
+
+
+def ring_line(w, n, steps, warmup, job_ms, ring_ms_rank0, fused_ms, e2e_ms, h2d, d2h, clocks, peak, peak_src):
+    """The JSON line of the ring mode: the whole problem's FLOPs over the slowest
+    rank's step time (strong scaling)."""
+    value = w.flops / (job_ms * 1e-3) / 1e12
+    cfg = config_of(w)
+    cfg.update(N=n, ranks="one process per GPU, CUDA IPC slot buffers, gloo host barrier",
+               step="ring forward of every rank: fill own slot, one host barrier, one cooperative launch "
+                    "fetching the other ranks' K/V blocks over NVLink while computing, merge of the parts")
+    achieved = w.flops / n / (ring_ms_rank0 * 1e-3) / 1e12
+    return {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": n, "steps": steps, "warmup": warmup,
+        "ms_per_step": job_ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": cfg,
+        "roofline": {"kernel": "attn_fwd_kernel<128,true> ring launch + merge, rank 0", "bound": "tensor",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": f"{peak_src} bf16_tflops (burst)", "ms": ring_ms_rank0},
+        "components": {"fused_one_gpu_ms": fused_ms,
+                       "ring_overhead_vs_fused_share": None if not fused_ms else job_ms / (fused_ms / n) - 1.0,
+                       "note": "fused_one_gpu_ms: the one-GPU fused forward of the whole problem on rank 0's GPU; "
+                               "the overhead compares the ring step with 1/N of it"},
+        "e2e": {"value": w.flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "note": "every rank uploads its own Q/K/V chunk from pinned memory and reads back its O and lse "
+                        "each step; bytes summed over the ranks"},
+        "gpu_launches": 2 * n * steps,
+        "clocks": clocks,
+    }
+
+
+def ring_main(args, ws, rank, local):
+    """bench.py --gpus N under torchrun: the ring over N GPUs (see the module doc)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import context_long_sequence_cp_b200 as cp
+    from context_long_sequence_cp_b200 import ring as R
+    from workloads import WORKLOADS, make_qkv
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    w = WORKLOADS[args.workload]
+    if args.layout:
+        w = w.with_layout(args.layout)
+    if w.layout == "ulysses":
+        raise SystemExit("the ring mode runs the contiguous and zigzag layouts")
+    B, H, S, D, N = w.B, w.H, w.S, w.D, ws
+    plan = cp.Plan(B, H, S, D, N, w.causal, w.layout)
+    nat = make_qkv(w)
+    # this rank's chunk in the layout's local order, through the library's layout map
+    chunks = []
+    for x in nat:
+        y = cp.layout_permute(plan, x.to(dev), 0).view(N, B, S // N, H, D)
+        chunks.append(y[rank].contiguous())
+        del y
+    q, k, v = chunks
+    ring = R.IpcRing(plan)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
+
+    def barrier():
+        dist.barrier(group=ring.group)
+        torch.cuda.synchronize(dev)
+
+    def events():
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        class _E:
+            def __init__(self, e):
+                self.e = e
+
+            def record(self):
+                self.e.record(stream)
+
+            def elapsed_time(self, other):
+                return self.e.elapsed_time(other.e)
+        return _E(a), _E(b)
+
+    with ClockSampler(local) as clk:
+        t0 = time.time()
+        local_ms = timed_ring_steps(lambda: ring.forward(q, k, v, stream), barrier, events, args.steps, args.warmup)
+        clocks = clk.window(t0, time.time())
+        st = cp.check(plan)
+        if st != 0:
+            raise RuntimeError(f"ring forward failed on rank {rank}: {cp.status_string(st)}")
+        job_ms, _ = job_throughput(local_ms, w.flops / N, ws, dev)
+        # end to end: each rank's chunk from pinned host memory, result read back
+        q_p, k_p, v_p = (x.cpu().pin_memory() for x in (q, k, v))
+        o_p = torch.empty_like(q_p).pin_memory()
+        l_p = torch.empty(B * (S // N) * H, dtype=torch.float32).pin_memory()
+        qi, ki, vi = (torch.empty_like(x) for x in (q, k, v))
+
+        def e2e_step():
+            qi.copy_(q_p, non_blocking=True)
+            ki.copy_(k_p, non_blocking=True)
+            vi.copy_(v_p, non_blocking=True)
+            o, lse = ring.forward(qi, ki, vi, stream)
+            o_p.copy_(o.view(o_p.shape), non_blocking=True)
+            l_p.copy_(lse, non_blocking=True)
+
+        e_local = timed_ring_steps(e2e_step, barrier, events, max(3, min(args.steps, 10)), 2)
+        e_ms, _ = job_throughput(e_local, w.flops / N, ws, dev)
+        # the one-GPU fused forward of the whole problem, on rank 0's GPU only
+        fused_ms = None
+        if rank == 0:
+            p1 = cp.Plan(B, H, S, D, w.N, w.causal, w.layout)
+            full = [cp.layout_permute(p1, x.to(dev), 0) for x in nat]
+            o1 = torch.empty_like(full[0])
+            l1 = torch.empty(B, H, S, dtype=torch.float32, device=dev)
+            legs = Legs(torch, dev, stream, clk)
+            fused_ms, _ = legs.back_to_back(lambda: cp.attn_fwd(p1, *full, o=o1, lse=l1), 10)
+            del full, o1, l1
+            p1.close()
+        barrier()
+    if rank == 0:
+        per_rank = q.numel() * 2
+        line = ring_line(w, N, args.steps, args.warmup, job_ms, local_ms, fused_ms, e_ms, 3 * per_rank * N,
+                         (per_rank + B * (S // N) * H * 4) * N, clocks, float(peaks["bf16_tflops"]), peak_src)
+        print(json.dumps(line), flush=True)
+    ring.close()
+    plan.close()
+    dist.destroy_process_group()
+    return 0
+
+
 def main():
     from workloads import WORKLOADS
     ap = argparse.ArgumentParser()
@@ -530,6 +682,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS),
                     help="workload of the step (default: the 32k zigzag headline)")
     ap.add_argument("--layout", default=None, help="override the workload's layout (long_128k: contiguous|zigzag)")
+    ap.add_argument("--mode", choices=["ring", "replica"], default="ring",
+                    help="under torchrun: the ring over the N GPUs (default) or N independent replicas")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-components", action="store_true", help="skip the component legs (32k workload)")
     ap.add_argument("--profile", choices=["attn", "merge", "permute", "rope", "sp", "bwd", "ring"], default=None,
@@ -539,6 +693,9 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    ws, rank, local = dist_env()
+    if ws > 1 and args.mode == "ring" and not args.profile:
+        return ring_main(args, ws, rank, local)
 
     import torch
     import torch.distributed as dist
