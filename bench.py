@@ -361,11 +361,12 @@ def profile_mode(args, cp, torch, plan, w, dev, q, k, v, qz, kz, vz, oz, lse, q_
         rslots_v[0].copy_(vz[0])
         r_arr = torch.zeros(N, dtype=torch.int32, device=dev)
         r_src = ([kz[j].data_ptr() for j in range(N)], [vz[j].data_ptr() for j in range(N)])
+        r_ws = torch.empty(plan.ring_merged_workspace_bytes(), dtype=torch.uint8, device=dev)
     if args.profile == "sp":
         sp = sp_inputs(torch, dev, S)
     for _ in range(args.warmup + args.steps):
         if args.profile == "ring":
-            cp.attn_fwd_ring(plan, 0, qz[0], rslots_k, rslots_v, r_src[0], r_src[1], r_arr)
+            cp.attn_fwd_ring_merged(plan, 0, qz[0], rslots_k, rslots_v, r_src[0], r_src[1], r_arr, workspace=r_ws)
         elif args.profile == "bwd":
             cp.attn_bwd(plan, qz, kz, vz, oz, lse, dod, gq, gk, gv, bws)
         elif args.profile == "attn":
@@ -493,9 +494,15 @@ def ring_components(cp, torch, plan, w, dev, stream, legs, qz, kz, vz, oz, att_m
         if cp.check(plan) != 0 or not ring_err <= 2e-2:
             raise RuntimeError(f"ring rank 0 disagrees with the fused forward: {ring_err}")
     ring_ms, c = legs.flushed(lambda: rr.forward(q0, kz[0], vz[0], stream), 7)
-    op_r, lp_r = rr.o_parts, rr.lse_parts
+    P = plan.ring_parts()
+    op_r = torch.empty(P, plan.rows // N, D, dtype=torch.float32, device=dev)
+    lp_r = torch.empty(P, plan.rows // N, dtype=torch.float32, device=dev)
+    mws = torch.empty(plan.ring_merged_workspace_bytes(), dtype=torch.uint8, device=dev)
 
-    def launch_only():
+    def launch_only():          # blocks resident, merge on chip
+        cp.attn_fwd_ring_merged(plan, 0, q0, kz, vz, o=ro, lse=rl, workspace=mws, stream=stream)
+
+    def launch_and_merge():     # blocks resident, tail partial + merge kernel
         cp.attn_fwd_ring(plan, 0, q0, kz, vz, o_parts=op_r, lse_parts=lp_r, stream=stream)
         cp.merge_partials(op_r, lp_r, o_out=ro, lse_out=rl)
 
@@ -508,21 +515,25 @@ def ring_components(cp, torch, plan, w, dev, stream, legs, qz, kz, vz, oz, att_m
         cp.merge_partials(op_s, lp_s, o_out=ro, lse_out=rl)
 
     ring_launch_ms, _ = legs.flushed(launch_only, 7)
+    ring_unmerged_ms, _ = legs.flushed(launch_and_merge, 7)
     ring_steps_ms, _ = legs.flushed(step_launches, 7)
     if cp.check(plan) != 0:
         raise RuntimeError("ring runs failed")
     rr.close()
     return {
         "ring_rank_ms": ring_ms, "ring_rank_tflops": w.flops / N / (ring_ms * 1e-3) / 1e12,
-        "ring_rank_launch_only_ms": ring_launch_ms, "ring_rank_step_launches_ms": ring_steps_ms,
+        "ring_rank_launch_only_ms": ring_launch_ms, "ring_rank_launch_then_merge_ms": ring_unmerged_ms,
+        "ring_rank_step_launches_ms": ring_steps_ms,
         "ring_rank_fused_share_ms": att_ms / N, "ring_overhead_vs_fused_share": ring_ms / (att_ms / N) - 1.0,
         "ring_fetch_cost": ring_ms / ring_launch_ms - 1.0, "ring_fetch_bytes": (N - 1) * 2 * blk,
         "ring_parts": plan.ring_parts(), "ring_clock": c,
         "ring_note": f"rank 0 of {N} on one GPU: fill + one cooperative launch whose copy warps fetch the "
                      f"other {N - 1} K/V blocks ({(N - 1) * 2 * blk >> 20} MiB; here from local HBM, on N "
-                     "GPUs over NVLink) while its units compute, + merge of the parts; launch_only = blocks "
-                     "resident; step_launches = one launch per ring step; fused_share = the fused launch / N; "
-                     "L2 flushed before each call",
+                     "GPUs over NVLink) while its units compute, the tail unit of each query tile merging the "
+                     "first-phase partials on chip; launch_only = blocks resident; launch_then_merge = blocks "
+                     "resident, tail partial + merge kernel instead of the on-chip merge; step_launches = one "
+                     "launch per ring step + merge; fused_share = the fused launch / N; L2 flushed before each "
+                     "call",
     }
 
 
@@ -552,13 +563,13 @@ def ring_line(w, n, steps, warmup, job_ms, ring_ms_rank0, fused_ms, e2e_ms, h2d,
     cfg = config_of(w)
     cfg.update(N=n, ranks="one process per GPU, CUDA IPC slot buffers, gloo host barrier",
                step="ring forward of every rank: fill own slot, one host barrier, one cooperative launch "
-                    "fetching the other ranks' K/V blocks over NVLink while computing, merge of the parts")
+                    "fetching the other ranks' K/V blocks over NVLink while computing and merging on chip")
     achieved = w.flops / n / (ring_ms_rank0 * 1e-3) / 1e12
     return {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": n, "steps": steps, "warmup": warmup,
         "ms_per_step": job_ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic", "config": cfg,
-        "roofline": {"kernel": "attn_fwd_kernel<128,true> ring launch + merge, rank 0", "bound": "tensor",
+        "roofline": {"kernel": "attn_fwd_kernel<128,true> merged ring launch, rank 0", "bound": "tensor",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "traffic": None, "peak_source": f"{peak_src} bf16_tflops (burst)", "ms": ring_ms_rank0},
         "components": {"fused_one_gpu_ms": fused_ms,
@@ -569,7 +580,7 @@ def ring_line(w, n, steps, warmup, job_ms, ring_ms_rank0, fused_ms, e2e_ms, h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "note": "every rank uploads its own Q/K/V chunk from pinned memory and reads back its O and lse "
                         "each step; bytes summed over the ranks"},
-        "gpu_launches": 2 * n * steps,
+        "gpu_launches": n * steps,
         "clocks": clocks,
     }
 
@@ -720,13 +731,13 @@ def main():
     if uly:   # the inputs are the N sequence shards (the natural tensor split along S)
         q_h, k_h, v_h = (x.reshape(B, N, S // N, H, D).transpose(0, 1).contiguous() for x in (q_h, k_h, v_h))
     q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
+    nws = plan.workspace_bytes(False)   # Ulysses head groups, or the split forward of a short problem
+    ws_buf = torch.empty(nws, dtype=torch.uint8, device=dev) if nws > 0 else None
     if uly:
         qz, kz, vz = q, k, v
         oz = torch.empty_like(q)
-        ws_buf = torch.empty(plan.workspace_bytes(False), dtype=torch.uint8, device=dev)
     else:
         qz, kz, vz, oz = (torch.empty_like(q).view(N, B, S // N, H, D) for _ in range(4))
-        ws_buf = None
     o = torch.empty_like(q)
     lse = torch.empty(B, H, S, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -741,7 +752,7 @@ def main():
                         vi if vi is not None else v, o=oi if oi is not None else o,
                         lse=li if li is not None else lse, workspace=ws_buf)
         else:
-            cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=li if li is not None else lse)
+            cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=li if li is not None else lse, workspace=ws_buf)
 
     def step(qi=q, ki=k, vi=v, oi=o, li=lse):
         if uly:
@@ -750,7 +761,7 @@ def main():
         cp.layout_permute(plan, qi, 0, out=qz)
         cp.layout_permute(plan, ki, 0, out=kz)
         cp.layout_permute(plan, vi, 0, out=vz)
-        cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=li)
+        cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=li, workspace=ws_buf)
         cp.layout_permute(plan, oz, 1, out=oi)
 
     launches_per_step = 5   # 3 layout maps + attention + inverse map (Ulysses: the same inside cp_attn_fwd)
@@ -810,7 +821,8 @@ def main():
             att_kernel = "cp_attn_fwd (Ulysses: 3 maps + attn_fwd_kernel<128,false> + 1 map)"
         else:
             att_fn = attention
-            att_kernel = f"attn_fwd_kernel<{D},false>"
+            att_kernel = f"attn_fwd_kernel<{D},false>" if ws_buf is None else \
+            f"attn_fwd_kernel<{D},true> (split walks of a short problem, merged on chip)"
         att, att_clock = (legs.flushed(att_fn, reps) if small else legs.back_to_back(att_fn, reps))
         att_tflops = w.flops / (att * 1e-3) / 1e12
         st = cp.check(plan)

@@ -544,6 +544,95 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tl = (PARTIAL ? item_qp(w) : w.qp) * kPair + wg * kTile + row;
       const int64_t row_id = (static_cast<int64_t>(w.rb - p.q_rb0) * g.T + tl) * g.Hh + w.h +
                              (PARTIAL && p.unit_steps ? min(unit_t0(w), p.unit_split) * p.part_rows : 0);
+      // Merged unit launch: the query tile's completion count (row blocks counted
+      // from q_rb0: one rank's B blocks in a ring launch, all of them otherwise).
+      const bool merged = PARTIAL && p.unit_steps && p.merge_done != nullptr;
+      const int rbl = w.rb - p.q_rb0;
+      int* const done = merged ? p.merge_done + (static_cast<int64_t>(rbl) * g.Hh + w.h) * p.merge_tiles +
+                                     (item_qp(w) * 2 + wg)
+                               : nullptr;
+      if (merged && unit_t0(w) >= p.unit_split) {
+        // ------------------------------------------------------ tail unit: merge
+        // Own partial (O / l, lse) as the partial path would write it, then the
+        // first-phase partials of this query tile once all of them are written,
+        // combined in the merge kernel's order (parts 0 .. split - 1, own last)
+        // and arithmetic, so the result equals partials + merge bit for bit.
+        float inv = 0.f, lse_own = -INFINITY;
+        if (ntile > 0) {
+          ok = mbar_wait(smem_addr(&sm.o_done[wg]), od_cnt & 1, ctl);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ++od_cnt;
+          tc_fence_after();
+          inv = l_run > 0.f ? 1.f / l_run : 0.f;
+          lse_own = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+        }
+        ok = count_wait(done, 4 * p.unit_split, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const int64_t prow = (static_cast<int64_t>(rbl) * g.T + tl) * g.Hh + w.h;
+        float M = -INFINITY;
+        if (valid) {
+          for (int t = 0; t < p.unit_split; ++t) M = fmaxf(M, ld_cg_f(p.lse_part + t * p.part_rows + prow));
+          M = fmaxf(M, lse_own);
+        }
+        const float Ms = M == -INFINITY ? 0.f : M;
+        float tot = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 16) {
+          uint32_t o[16];
+          if (ntile > 0) tmem_ld16(tO + c, o);   // uniform over the warpgroup
+          if (valid) {
+            float acc[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+            for (int t = 0; t <= p.unit_split; ++t) {
+              const bool own = t == p.unit_split;
+              const float wt = expf((own ? lse_own : ld_cg_f(p.lse_part + t * p.part_rows + prow)) - Ms);
+              if (wt != 0.f) {
+                if (own) {
+#pragma unroll
+                  for (int j = 0; j < 16; ++j) acc[j] = fmaf(wt, __uint_as_float(o[j]) * inv, acc[j]);
+                } else {
+                  const float* src = p.o_part + (t * p.part_rows + prow) * D + c;
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) {
+                    const float4 v = ld_cg_f4(src + 4 * j);
+                    acc[4 * j] = fmaf(wt, v.x, acc[4 * j]);
+                    acc[4 * j + 1] = fmaf(wt, v.y, acc[4 * j + 1]);
+                    acc[4 * j + 2] = fmaf(wt, v.z, acc[4 * j + 2]);
+                    acc[4 * j + 3] = fmaf(wt, v.w, acc[4 * j + 3]);
+                  }
+                }
+                if (c == 0) tot += wt;
+              }
+            }
+            const float it = tot > 0.f ? 1.f / tot : 0.f;
+            uint4* dst = reinterpret_cast<uint4*>(p.o_final + prow * D + c);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              uint4 u;
+              u.x = pack_bf16x2(acc[8 * j + 0] * it, acc[8 * j + 1] * it);
+              u.y = pack_bf16x2(acc[8 * j + 2] * it, acc[8 * j + 3] * it);
+              u.z = pack_bf16x2(acc[8 * j + 4] * it, acc[8 * j + 5] * it);
+              u.w = pack_bf16x2(acc[8 * j + 6] * it, acc[8 * j + 7] * it);
+              dst[j] = u;
+            }
+          }
+        }
+        if (valid) {
+          const float lse = M == -INFINITY ? -INFINITY : Ms + logf(tot);
+          if (p.lse_final != nullptr) {
+            p.lse_final[prow] = lse;   // rows in the partials' order
+          } else if (p.lse != nullptr) {
+            // natural [B][H][S] order, as the fused forward writes it
+            const int64_t li = (static_cast<int64_t>(bv % p.lse_B) * p.lse_H + (bv / p.lse_B) * g.Hh + w.h) *
+                                   p.lse_S + gq;
+            p.lse[li] = lse;
+          }
+        }
+        continue;
+      }
       if (ntile > 0) {
         ok = mbar_wait(smem_addr(&sm.o_done[wg]), od_cnt & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
@@ -602,6 +691,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             p.lse[li] = -INFINITY;
           }
         }
+      }
+      if (merged) {
+        // First-phase unit of a merged ring launch: its partial rows are written;
+        // publish them to the query tile's tail unit (one count per warp).
+        chunk_stores_fence();
+        __syncwarp();
+        if (lane == 0) red_release_add(done, 1);
       }
     }
   }
@@ -678,7 +774,9 @@ cudaError_t launch_impl(const FwdLaunch& L, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = (PARTIAL && L.params.pull_chunks > 0) ? 1 : 0;
+  // A merged ring launch is cooperative too: tail units wait for first-phase
+  // units of other CTAs.
+  cfg.numAttrs = (PARTIAL && (L.params.pull_chunks > 0 || L.params.merge_done != nullptr)) ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, L.tm_q, L.tm_k, L.tm_v, L.params);
 }
 

@@ -168,6 +168,11 @@ __device__ __forceinline__ void red_release_add(int* count, int v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(count), "r"(v) : "memory");
 }
 
+// Loads of data other CTAs of this kernel wrote (ordered after an acquire of
+// their release count): cached in L2 only, never in a possibly stale L1.
+__device__ __forceinline__ float4 ld_cg_f4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ float ld_cg_f(const float* p) { return __ldcg(p); }
+
 // 16-byte streaming load (read-only for the kernel's lifetime, no L1 allocation)
 // and store.
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
