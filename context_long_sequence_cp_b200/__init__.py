@@ -30,7 +30,6 @@ SIGNATURES = {
     "cp_attn_plan_destroy": (_I, [_P]),
     "cp_attn_plan_tile_counts": (_I64, [_P, _P]),
     "cp_attn_plan_num_items": (_I64, [_P]),
-    "cp_attn_plan_split_units": (_I64, [_P, _P]),
     "cp_attn_plan_cta_loads": (_I64, [_P, _P]),
     "cp_attn_bwd": (_I, [_P] * 12),
     "cp_sp_rs_dropout_add_ln": (_I, [_P, _I, _I64, _I, _P, ctypes.c_float, _P, _P, _P, ctypes.c_float, _P, _P, _P]),
@@ -53,8 +52,6 @@ SIGNATURES = {
     "cp_attn_ring_num_parts": (_I, [_P]),
     "cp_attn_fwd_ring": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "cp_attn_fwd_ring_external": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P]),
-    "cp_attn_ring_merged_workspace_bytes": (_SZ, [_P]),
-    "cp_attn_fwd_ring_merged": (_I, [_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "cp_attn_ring_schedule": (_I64, [_P, _I, _I, _P, _P]),
     "cp_ring_buffer_alloc": (_I, [_SZ, ctypes.POINTER(_P)]),
     "cp_ring_buffer_free": (_I, [_P]),
@@ -148,14 +145,6 @@ class Plan:
     def num_items(self) -> int:
         return int(lib().cp_attn_plan_num_items(self._h))
 
-    def split_units(self):
-        """(units, first-phase steps) of the split forward of a short problem; (0, 0) when not split."""
-        st = ctypes.c_int(0)
-        n = int(lib().cp_attn_plan_split_units(self._h, ctypes.byref(st)))
-        if n < 0:
-            raise CpAttnError("cp_attn_plan_split_units", n)
-        return n, int(st.value)
-
     def bwd_pairs(self):
         """(key-tile walk pairs, query-tile walk pairs) of the backward, per (batch, head)."""
         kv, qq = ctypes.c_int64(0), ctypes.c_int64(0)
@@ -202,10 +191,6 @@ class Plan:
         rows = [tuple(items[5 * i:5 * i + 5]) for i in range(n)]
         n_cta = max(r[4] for r in rows) + 1 if rows else 0
         return rows, list(loads)[:n_cta]
-
-    def ring_merged_workspace_bytes(self) -> int:
-        """Workspace of the merged one-launch ring forward (``cp_attn_fwd_ring_merged``)."""
-        return int(lib().cp_attn_ring_merged_workspace_bytes(self._h))
 
     def workspace_bytes(self, with_partials: bool = False) -> int:
         return int(lib().cp_attn_workspace_bytes(self._h, int(with_partials)))
@@ -283,28 +268,6 @@ def attn_fwd_ring(plan: Plan, rank: int, q, k_all, v_all, pull_k=None, pull_v=No
                                   as_ptr(pv), None if arrived is None else _vp_of(arrived), _ptr(o_parts),
                                   _ptr(lse_parts), _stream(stream)))
     return o_parts, lse_parts
-
-
-def attn_fwd_ring_merged(plan: Plan, rank: int, q, k_all, v_all, pull_k=None, pull_v=None, arrived=None, o=None,
-                         lse=None, workspace=None, stream=None):
-    """``cp_attn_fwd_ring_merged``: the rank's rows of full attention from one
-    launch (arguments as ``attn_fwd_ring``). Returns (o bf16 [B, S/N, H, D],
-    lse fp32 [rows])."""
-    T = plan.S // plan.N
-    if o is None:
-        o = torch.empty(plan.B, T, plan.H, plan.D, dtype=torch.bfloat16, device=q.device)
-    if lse is None:
-        lse = torch.empty(plan.B * T * plan.H, dtype=torch.float32, device=q.device)
-    if workspace is None:
-        workspace = torch.empty(plan.ring_merged_workspace_bytes(), dtype=torch.uint8, device=q.device)
-    pk = None if pull_k is None else (ctypes.c_void_p * len(pull_k))(*[int(x) for x in pull_k])
-    pv = None if pull_v is None else (ctypes.c_void_p * len(pull_v))(*[int(x) for x in pull_v])
-    as_ptr = lambda a: None if a is None else ctypes.cast(a, ctypes.c_void_p)
-    _check("cp_attn_fwd_ring_merged",
-           lib().cp_attn_fwd_ring_merged(plan.handle, int(rank), _ptr(q), _vp_of(k_all), _vp_of(v_all), as_ptr(pk),
-                                         as_ptr(pv), None if arrived is None else _vp_of(arrived), _ptr(o), _ptr(lse),
-                                         _ptr(workspace), _stream(stream)))
-    return o, lse
 
 
 def attn_fwd_ring_external(plan: Plan, rank: int, q, k_all, v_all, arrived, o_parts=None, lse_parts=None,

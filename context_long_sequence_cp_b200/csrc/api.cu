@@ -86,17 +86,6 @@ struct cp_attn_plan_s {
   };
   int sms = kDefaultSmCountPlan;
   std::vector<RingRank> ring;
-  // Short problems (fewer work items than a few per SM): the fused forward runs
-  // each pair's walk as units over ring steps (one per step before split_steps,
-  // then one tail unit over the rest that merges the others' partials on chip),
-  // giving the CTAs several times more, smaller pieces to balance.
-  int split_steps = 0;                // 0: the plan does not split
-  std::vector<WorkItem> split_units;
-  std::vector<int> split_cta_begin;
-  std::vector<int64_t> split_cta_load;
-  int split_n_cta = 0;
-  WorkItem* d_split_units = nullptr;
-  int* d_split_cta_begin = nullptr;
 };
 
 namespace {
@@ -211,52 +200,6 @@ void schedule_items(cp_attn_plan_s* p, int n_cta) {
   p->n_cta = assign_greedy(p->items, cost, n_cta, p->cta_begin, p->cta_load);
 }
 
-// Items per SM below which a plan's fused forward splits its walks into units.
-constexpr int kSplitItemsPerSm = 4;
-
-// Units of the split forward over the whole view: per (rank, batch, query-tile
-// pair, head) one unit per ring step t < split and one tail unit over [split,
-// NR), ordered phase-major (every first-phase unit precedes every tail unit in
-// each CTA's list, so a tail unit's wait for its first-phase units always ends),
-// longest first within a phase, then assigned by the greedy rule.
-void build_split(cp_attn_plan_s* p, int n_cta) {
-  const Geometry& g = p->g;
-  const int split = g.NR <= 2 ? 1 : (g.NR + 1) / 2;
-  struct U {
-    WorkItem w;
-    int64_t cost;
-    int phase;
-  };
-  std::vector<U> us;
-  for (int r = 0; r < g.NR; ++r)
-    for (int b = 0; b < g.B; ++b)
-      for (int qp = 0; qp < p->npairs; ++qp) {
-        const int* off = p->step_off.data() + static_cast<size_t>(r * p->npairs + qp) * (g.NR + 1);
-        for (int h = 0; h < g.Hh; ++h) {
-          for (int t = 0; t < split; ++t) {
-            const int len = off[t + 1] - off[t];
-            us.push_back(U{WorkItem{r * g.B + b, h, pack_unit(qp, t, t + 1), len},
-                           2 * static_cast<int64_t>(len) + kItemOverheadHalfTiles, t});
-          }
-          const int len = off[g.NR] - off[split];
-          us.push_back(U{WorkItem{r * g.B + b, h, pack_unit(qp, split, g.NR), len},
-                         2 * static_cast<int64_t>(len) + kItemOverheadHalfTiles, split});
-        }
-      }
-  std::stable_sort(us.begin(), us.end(), [](const U& x, const U& y) {
-    if (x.phase != y.phase) return x.phase < y.phase;
-    return x.cost > y.cost;
-  });
-  p->split_units.clear();
-  std::vector<int64_t> cost;
-  for (const U& u : us) {
-    p->split_units.push_back(u.w);
-    cost.push_back(u.cost);
-  }
-  p->split_n_cta = assign_greedy(p->split_units, cost, n_cta, p->split_cta_begin, p->split_cta_load);
-  p->split_steps = split;
-}
-
 // Walks and schedules of the two backward kernels. A walk entry's class is
 // kFull when every (row, column) pair of the tile pair is allowed and both tiles
 // are whole; otherwise kMasked (the kernels then bound the allowed columns).
@@ -327,21 +270,6 @@ void free_bwd(cp_attn_plan_s::BwdSched& b) {
   b.d_cta_begin = nullptr;
   b.d_walk_off = nullptr;
   b.d_entries = nullptr;
-}
-
-bool upload_split(cp_attn_plan_s* p) {
-  const size_t ub = p->split_units.size() * sizeof(WorkItem), cb = p->split_cta_begin.size() * sizeof(int);
-  return cudaMalloc(&p->d_split_units, ub > 0 ? ub : sizeof(WorkItem)) == cudaSuccess &&
-         cudaMalloc(&p->d_split_cta_begin, cb) == cudaSuccess &&
-         (ub == 0 || cudaMemcpy(p->d_split_units, p->split_units.data(), ub, cudaMemcpyHostToDevice) == cudaSuccess) &&
-         cudaMemcpy(p->d_split_cta_begin, p->split_cta_begin.data(), cb, cudaMemcpyHostToDevice) == cudaSuccess;
-}
-
-void free_split(cp_attn_plan_s* p) {
-  if (p->d_split_units != nullptr) cudaFree(p->d_split_units);
-  if (p->d_split_cta_begin != nullptr) cudaFree(p->d_split_cta_begin);
-  p->d_split_units = nullptr;
-  p->d_split_cta_begin = nullptr;
 }
 
 int ensure_device(cp_attn_plan_s* p) {
@@ -514,77 +442,6 @@ PermuteArgs permute_args(const cp_attn_plan_s* p, int direction, int elem_bytes)
   return a;
 }
 
-// Layout of the merged ring launch's workspace: the first-phase partials (split
-// parts of rows x D fp32, then split x rows fp32 lse), then the completion
-// counts (B x H x 2 x query-tile pairs int32, one per query tile of every pair,
-// a ragged pair's empty second tile included), each piece 256-byte aligned.
-struct RingMergedWs {
-  size_t o_off, lse_off, done_off, bytes;
-};
-// row_blocks: B for one rank of a ring launch, NR * B for the whole view.
-RingMergedWs merged_ws(const cp_attn_plan_s* plan, int row_blocks, int parts_n) {
-  const Geometry& g = plan->g;
-  const size_t rows = static_cast<size_t>(row_blocks) * g.T * g.Hh;
-  const size_t parts = static_cast<size_t>(parts_n);
-  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-  RingMergedWs w;
-  w.o_off = 0;
-  w.lse_off = up(parts * rows * plan->D * 4);
-  w.done_off = w.lse_off + up(parts * rows * 4);
-  w.bytes = w.done_off + up(static_cast<size_t>(row_blocks) * g.Hh * 2 * ((g.T + kPair - 1) / kPair) * 4);
-  return w;
-}
-RingMergedWs ring_merged_ws(const cp_attn_plan_s* plan) { return merged_ws(plan, plan->g.B, ring_split(plan->g.NR)); }
-RingMergedWs split_ws(const cp_attn_plan_s* plan) {
-  return merged_ws(plan, plan->g.NR * plan->g.B, plan->split_steps);
-}
-
-// The split forward (plan->split_steps > 0) over the whole view, writing o and
-// lse like the fused launch.
-int launch_split(cp_attn_plan_s* p, const void* q, const void* k, const void* v, void* o, float* lse,
-                 void* workspace, cudaStream_t st) {
-  const Geometry& g = p->g;
-  FwdLaunch L;
-  std::memset(&L, 0, sizeof(L));
-  int rc;
-  if ((rc = encode_view(&L.tm_q, q, g, p->D)) != CP_OK) return rc;
-  if ((rc = encode_view(&L.tm_k, k, g, p->D)) != CP_OK) return rc;
-  if ((rc = encode_view(&L.tm_v, v, g, p->D)) != CP_OK) return rc;
-  const RingMergedWs w = split_ws(p);
-  char* ws = static_cast<char*>(workspace);
-  FwdParams& P = L.params;
-  P.g = g;
-  P.t_begin = 0;
-  P.t_end = g.NR;
-  P.scale_log2 = p->scale * 1.4426950408889634f;
-  P.items = p->d_split_units;
-  P.n_items = static_cast<int>(p->split_units.size());
-  P.cta_begin = p->d_split_cta_begin;
-  P.n_cta = p->split_n_cta;
-  P.step_off = p->d_step_off;
-  P.entries = p->d_entries;
-  P.npairs = p->npairs;
-  P.lse = lse;
-  P.lse_B = p->lse_B;
-  P.lse_H = p->lse_H;
-  P.lse_S = p->lse_S;
-  P.o_part = reinterpret_cast<float*>(ws + w.o_off);
-  P.lse_part = reinterpret_cast<float*>(ws + w.lse_off);
-  P.unit_steps = 1;
-  P.unit_split = p->split_steps;
-  P.part_rows = static_cast<int64_t>(g.NR) * g.B * g.T * g.Hh;
-  P.merge_done = reinterpret_cast<int*>(ws + w.done_off);
-  P.merge_tiles = 2 * p->npairs;
-  P.o_final = static_cast<__nv_bfloat16*>(o);
-  P.lse_final = nullptr;   // lse in natural order through P.lse
-  P.status = p->d_status;
-  P.wait_limit_ns = kWaitLimitNs;
-  if (cudaMemsetAsync(P.merge_done, 0, sizeof(int) * static_cast<size_t>(g.NR) * g.B * g.Hh * P.merge_tiles, st) !=
-      cudaSuccess)
-    return CP_ERR_CUDA;
-  return launch_attn_fwd(L, p->D, true, st) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
-}
-
 }  // namespace
 
 extern "C" {
@@ -691,9 +548,6 @@ int cp_attn_plan(cp_attn_plan_t* out, int B, int H, int S, int D, int N, int cau
   p->ring.resize(layout == CP_LAYOUT_ULYSSES ? 0 : g.NR);
   schedule_items(p, sms);
   if (layout != CP_LAYOUT_ULYSSES) build_bwd(p, sms);
-  if (layout != CP_LAYOUT_ULYSSES && g.NR >= 2 && g.NR <= 255 &&
-      p->items.size() < static_cast<size_t>(kSplitItemsPerSm) * sms)
-    build_split(p, sms);
   if (have_device) {
     const size_t bytes = p->items.size() * sizeof(WorkItem);
     const size_t off_bytes = p->step_off.size() * sizeof(int);
@@ -710,12 +564,10 @@ int cp_attn_plan(cp_attn_plan_t* out, int B, int H, int S, int D, int N, int cau
               (ent_bytes == 0 ||
                cudaMemcpy(p->d_entries, p->entries.data(), ent_bytes, cudaMemcpyHostToDevice) == cudaSuccess) &&
               cudaMemset(p->d_status, 0, sizeof(int)) == cudaSuccess &&
-              (layout == CP_LAYOUT_ULYSSES || (upload_bwd(p->bwd_kv) && upload_bwd(p->bwd_q))) &&
-              (p->split_steps == 0 || upload_split(p));
+              (layout == CP_LAYOUT_ULYSSES || (upload_bwd(p->bwd_kv) && upload_bwd(p->bwd_q)));
     if (!ok) {
       free_bwd(p->bwd_kv);
       free_bwd(p->bwd_q);
-      free_split(p);
       cudaFree(p->d_items);
       cudaFree(p->d_cta_begin);
       p->d_cta_begin = nullptr;
@@ -740,7 +592,6 @@ int cp_attn_plan_destroy(cp_attn_plan_t plan) {
   if (plan->d_cta_begin != nullptr) cudaFree(plan->d_cta_begin);
   free_bwd(plan->bwd_kv);
   free_bwd(plan->bwd_q);
-  free_split(plan);
   for (auto& rr : plan->ring) free_ring(rr);
   if (plan->d_status != nullptr) cudaFree(plan->d_status);
   if (plan->d_step_off != nullptr) cudaFree(plan->d_step_off);
@@ -762,12 +613,6 @@ int64_t cp_attn_plan_tile_counts(cp_attn_plan_t plan, int64_t* per_rank) {
 int64_t cp_attn_plan_num_items(cp_attn_plan_t plan) {
   if (plan == nullptr) return CP_ERR_INVALID_ARG;
   return static_cast<int64_t>(plan->items.size());
-}
-
-int64_t cp_attn_plan_split_units(cp_attn_plan_t plan, int* split_steps) {
-  if (plan == nullptr) return CP_ERR_INVALID_ARG;
-  if (split_steps != nullptr) *split_steps = plan->split_steps;
-  return static_cast<int64_t>(plan->split_units.size());
 }
 
 size_t cp_attn_bwd_workspace_bytes(cp_attn_plan_t plan) {
@@ -859,7 +704,6 @@ size_t cp_attn_workspace_bytes(cp_attn_plan_t plan, int with_partials) {
   if (plan == nullptr) return 0;
   if (plan->layout == CP_LAYOUT_ULYSSES && !with_partials)
     return 4 * static_cast<size_t>(plan->B) * plan->S * plan->H * plan->D * 2;
-  if (plan->split_steps > 0 && !with_partials) return split_ws(plan).bytes;
   return 0;
 }
 
@@ -872,11 +716,8 @@ int cp_attn_fwd(cp_attn_plan_t plan, const void* q, const void* k, const void* v
   int rc = ensure_device(plan);
   if (rc != CP_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (plan->layout != CP_LAYOUT_ULYSSES) {
-    if (plan->split_steps > 0 && workspace != nullptr && plan->d_split_units != nullptr)
-      return launch_split(plan, q, k, v, o, lse, workspace, st);
+  if (plan->layout != CP_LAYOUT_ULYSSES)
     return launch_view(plan, plan->g, q, k, v, o, lse, nullptr, nullptr, 0, plan->g.NR, false, st);
-  }
 
   if (workspace == nullptr) return CP_ERR_WORKSPACE;
   const size_t tensor = static_cast<size_t>(plan->B) * plan->S * plan->H * plan->D * 2;
@@ -1020,11 +861,9 @@ namespace {
 // kernel's copy warps fetch the other blocks and count their chunks in arrived),
 // external (arrived[j] >= 1 is set by the caller's own transfer) and resident
 // (arrived NULL: every slot already holds its block, no wait).
-// Merged launches (o_final not NULL) take their first-phase partials and the
-// per-query-tile completion counts from `merge_ws` (cp_attn_ring_merged_workspace_bytes).
 int ring_launch(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all, const void* const* pull_k,
                 const void* const* pull_v, int* arrived, bool external, float* o_parts, float* lse_parts,
-                cp_stream_t stream, void* o_final = nullptr, float* lse_final = nullptr, int* merge_done = nullptr) {
+                cp_stream_t stream) {
   if (plan == nullptr || q == nullptr || k_all == nullptr || v_all == nullptr || o_parts == nullptr ||
       lse_parts == nullptr)
     return CP_ERR_INVALID_ARG;
@@ -1092,21 +931,12 @@ int ring_launch(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void*
   P.part_rows = static_cast<int64_t>(g.B) * g.T * g.Hh;
   P.arrived = arrived;
   P.arrive_target = pull ? P.pull_chunks : 1;
-  P.merge_done = merge_done;
-  P.merge_tiles = 2 * ((g.T + kPair - 1) / kPair);   // both query tiles of every pair, ragged ones included
-  P.o_final = static_cast<__nv_bfloat16*>(o_final);
-  P.lse_final = lse_final;
   P.status = plan->d_status;
   P.wait_limit_ns = kWaitLimitNs;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (pull && cudaMemsetAsync(arrived, 0, sizeof(int) * plan->N, st) != cudaSuccess) return CP_ERR_CUDA;
-  if (merge_done != nullptr &&
-      cudaMemsetAsync(merge_done, 0, sizeof(int) * static_cast<size_t>(g.B) * g.Hh * P.merge_tiles, st) != cudaSuccess)
-    return CP_ERR_CUDA;
   return launch_attn_fwd(L, plan->D, true, st) == cudaSuccess ? CP_OK : CP_ERR_CUDA;
 }
-
-
 
 }  // namespace
 
@@ -1121,36 +951,6 @@ int cp_attn_fwd_ring(cp_attn_plan_t plan, int rank, const void* q, void* k_all, 
 int cp_attn_fwd_ring_external(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all,
                               int* arrived, float* o_parts, float* lse_parts, cp_stream_t stream) {
   return ring_launch(plan, rank, q, k_all, v_all, nullptr, nullptr, arrived, true, o_parts, lse_parts, stream);
-}
-
-size_t cp_attn_ring_merged_workspace_bytes(cp_attn_plan_t plan) {
-  if (plan == nullptr || plan->layout == CP_LAYOUT_ULYSSES) return 0;
-  return ring_merged_ws(plan).bytes;
-}
-
-int cp_attn_fwd_ring_merged(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all,
-                            const void* const* pull_k, const void* const* pull_v, int* arrived, void* o, float* lse,
-                            void* workspace, cp_stream_t stream) {
-  if (plan == nullptr || o == nullptr || lse == nullptr || workspace == nullptr) return CP_ERR_INVALID_ARG;
-  if (plan->layout == CP_LAYOUT_ULYSSES) return CP_ERR_UNSUPPORTED;
-  if (!aligned16(o) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return CP_ERR_ALIGNMENT;
-  const RingMergedWs w = ring_merged_ws(plan);
-  char* ws = static_cast<char*>(workspace);
-  float* o_parts = reinterpret_cast<float*>(ws + w.o_off);
-  float* lse_parts = reinterpret_cast<float*>(ws + w.lse_off);
-  const int split = ring_split(plan->N);
-  if (split >= plan->N) {
-    // No tail phase (N <= 2): every step is a partial; merge them after the launch.
-    int rc = ring_launch(plan, rank, q, k_all, v_all, pull_k, pull_v, arrived, false, o_parts, lse_parts, stream);
-    if (rc != CP_OK) return rc;
-    const int64_t rows = static_cast<int64_t>(plan->g.B) * plan->g.T * plan->g.Hh;
-    return launch_merge(plan->N, rows, plan->D, o_parts, lse_parts, static_cast<__nv_bfloat16*>(o), lse,
-                        static_cast<cudaStream_t>(stream)) == cudaSuccess
-               ? CP_OK
-               : CP_ERR_CUDA;
-  }
-  return ring_launch(plan, rank, q, k_all, v_all, pull_k, pull_v, arrived, false, o_parts, lse_parts, stream, o, lse,
-                     reinterpret_cast<int*>(ws + w.done_off));
 }
 
 int cp_merge_partials(int num_parts, int64_t rows, int D, const float* o_parts, const float* lse_parts,

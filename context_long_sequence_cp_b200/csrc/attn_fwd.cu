@@ -121,7 +121,8 @@ __device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint32_t v_ad
 }
 
 // Exponentials of one 32-column chunk c of a score row, packed to bf16 pairs and
-// stored as 16 TMEM columns of P at tS + 16c; row-sum partials accumulate in ls.
+// stored as 16 TMEM columns of P at tS + 64 + 16c (over the scores of keys
+// 64-127, which are in registers by then); row-sum partials accumulate in ls.
 // The scaling x = s * scale - m runs two columns per instruction (f32x2).
 __device__ __forceinline__ void softmax_chunk(const float (&s)[kTile], int c, float sl2, float m_use,
                                               uint32_t tS, float (&ls)[8]) {
@@ -138,7 +139,7 @@ __device__ __forceinline__ void softmax_chunk(const float (&s)[kTile], int c, fl
     ls[j & 7] += e0 + e1;
     pk[j] = pack_bf16x2(e0, e1);
   }
-  tmem_st16(tS + c * 16, pk);
+  tmem_st16(tS + 64 + c * 16, pk);
 }
 
 // Maximum of the 64 scores s[32c .. 32c+63], four chains of 3-input maxima.
@@ -153,22 +154,6 @@ __device__ __forceinline__ float half_max(const float (&s)[kTile], int c) {
     m[k] = fmaxf(x, s[b + 15]);
   }
   return fmaxf(max3(m[0], m[1], m[2]), m[3]);
-}
-
-// Multiplies the 64 bf16 P values of keys 0-63 (TMEM columns tS .. tS+31, two
-// per column) by beta.
-__device__ __forceinline__ void rescale_p_half(uint32_t tS, float beta) {
-#pragma unroll
-  for (int c = 0; c < 32; c += 16) {
-    uint32_t v[16];
-    tmem_ld16(tS + c, v);
-#pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&v[q]);
-      v[q] = pack_bf16x2(__low2float(b) * beta, __high2float(b) * beta);
-    }
-    tmem_st16(tS + c, v);
-  }
 }
 
 }  // namespace
@@ -380,12 +365,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            issue_pv<D, 0, 4>(tO0, tS0, v_addr, acc0);
+            issue_pv<D, 0, 4>(tO0, tS0 + 64, v_addr, acc0);
             ok = mbar_wait(smem_addr(&sm.p_full[0][1]), p_cnt0 & 1, ctl);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            issue_pv<D, 4, 8>(tO0, tS0, v_addr, true);
+            issue_pv<D, 4, 8>(tO0, tS0 + 64, v_addr, true);
             ++p_cnt0;
             acc0 = true;
             if (e == last0) umma_commit_elect(smem_addr(&sm.o_done[0]));
@@ -401,12 +386,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            issue_pv<D, 0, 4>(tO1, tS1, v_addr, acc1);
+            issue_pv<D, 0, 4>(tO1, tS1 + 64, v_addr, acc1);
             ok = mbar_wait(smem_addr(&sm.p_full[1][1]), p_cnt1 & 1, ctl);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            issue_pv<D, 4, 8>(tO1, tS1, v_addr, true);
+            issue_pv<D, 4, 8>(tO1, tS1 + 64, v_addr, true);
             ++p_cnt1;
             acc1 = true;
             if (e == last1) umma_commit_elect(smem_addr(&sm.o_done[1]));
@@ -475,38 +460,52 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < kTile; ++j) s[j] = j < lim ? s[j] : -INFINITY;
         }
-        // Row max, then exponentials. The max of keys 0-63 comes first and their
-        // exponentials start at once; the max of keys 64-127 is computed while
-        // they run. Rescaling is lazy (only when the max grows by more than 2^8),
-        // so keys 64-127 rarely move the max; when they do, the stored P of keys
-        // 0-63 and its partial sums are scaled down to the new max before the
-        // MMA warp may read them.
+        // Exponentials, then the row max. Rescaling is lazy (the running max
+        // moves only when the scores exceed it by more than 2^8), so when every
+        // row of the warp has a running max, the exponentials of keys 0-63 start
+        // from it at once and the tile's own max is computed alongside them; a
+        // warp with a row still at -inf takes the max of keys 0-63 first. When
+        // the tile raises a row's max past the threshold (rare after a row's
+        // first tiles), P of keys 0-63 and its partial sums are recomputed from
+        // the scores with the new max before the MMA warp may read them.
         const float m_prev = m_run;
-        float m01 = half_max(s, 0);
-        bool resc = m01 * sl2 - m_run > kRescaleThreshold;   // false while both are -inf
-        if (resc) m_run = m01 * sl2;
+        const bool stale = __all_sync(0xffffffffu, m_run != -INFINITY);
+        // Stale path: the exponentials do not depend on m01, so its max chain
+        // overlaps them; it comes first only so the scores of keys 0-63 die early.
+        const float m01 = half_max(s, 0);
+        bool resc = false;
+        if (!stale) {
+          resc = m01 * sl2 - m_run > kRescaleThreshold;   // false while both are -inf
+          if (resc) m_run = m01 * sl2;
+        }
         float m_use = m_run == -INFINITY ? 0.f : m_run;
         float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         softmax_chunk(s, 0, sl2, m_use, tS, ls);
         softmax_chunk(s, 1, sl2, m_use, tS, ls);
         const float m23 = half_max(s, 2);
-        const bool resc_b = m23 * sl2 - m_run > kRescaleThreshold;
+        const float mt = stale ? fmaxf(m01, m23) : m23;
+        const bool resc_b = mt * sl2 - m_run > kRescaleThreshold;
         if (__any_sync(0xffffffffu, resc_b)) {
-          // Rare: keys 64-127 raise the max. P of keys 0-63 (32 packed columns)
-          // is scaled by 2^(m_use - m_use_new), exactly what recomputing it would
-          // give up to one more bf16 rounding.
-          float beta = 1.f;
           if (resc_b) {
-            // A row whose max was still -inf has all-zero P for keys 0-63.
-            beta = m_run == -INFINITY ? 0.f : ex2_approx(m_use - m23 * sl2);
-            m_run = m23 * sl2;
+            m_run = mt * sl2;
             m_use = m_run;
             resc = true;
           }
-          tmem_st_wait();   // the P just stored is read back
-          rescale_p_half(tS, beta);
+          // Recompute P of keys 0-63 with the (possibly) new max, from their
+          // scores, still intact in TMEM columns 0-63 (P is written over those
+          // of keys 64-127): exact, and no value computed from a stale max is
+          // ever published.
+          tmem_st_wait();
+          tmem_ld64(tS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]), *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+          if (cls == kMasked) {
+            const int lim = valid ? column_limit(g, entry_rank(cur), entry_tile(cur) * kTile, gq) : 0;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) ls[q] *= beta;
+            for (int j = 0; j < 64; ++j) s[j] = j < lim ? s[j] : -INFINITY;
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q) ls[q] = 0.f;
+          softmax_chunk(s, 0, sl2, m_use, tS, ls);
+          softmax_chunk(s, 1, sl2, m_use, tS, ls);
         }
         const float alpha = resc ? ex2_approx(m_prev - m_run) : 1.f;   // 0 when m_prev = -inf
         l_run *= alpha;
@@ -544,95 +543,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tl = (PARTIAL ? item_qp(w) : w.qp) * kPair + wg * kTile + row;
       const int64_t row_id = (static_cast<int64_t>(w.rb - p.q_rb0) * g.T + tl) * g.Hh + w.h +
                              (PARTIAL && p.unit_steps ? min(unit_t0(w), p.unit_split) * p.part_rows : 0);
-      // Merged unit launch: the query tile's completion count (row blocks counted
-      // from q_rb0: one rank's B blocks in a ring launch, all of them otherwise).
-      const bool merged = PARTIAL && p.unit_steps && p.merge_done != nullptr;
-      const int rbl = w.rb - p.q_rb0;
-      int* const done = merged ? p.merge_done + (static_cast<int64_t>(rbl) * g.Hh + w.h) * p.merge_tiles +
-                                     (item_qp(w) * 2 + wg)
-                               : nullptr;
-      if (merged && unit_t0(w) >= p.unit_split) {
-        // ------------------------------------------------------ tail unit: merge
-        // Own partial (O / l, lse) as the partial path would write it, then the
-        // first-phase partials of this query tile once all of them are written,
-        // combined in the merge kernel's order (parts 0 .. split - 1, own last)
-        // and arithmetic, so the result equals partials + merge bit for bit.
-        float inv = 0.f, lse_own = -INFINITY;
-        if (ntile > 0) {
-          ok = mbar_wait(smem_addr(&sm.o_done[wg]), od_cnt & 1, ctl);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          ++od_cnt;
-          tc_fence_after();
-          inv = l_run > 0.f ? 1.f / l_run : 0.f;
-          lse_own = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
-        }
-        ok = count_wait(done, 4 * p.unit_split, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        const int64_t prow = (static_cast<int64_t>(rbl) * g.T + tl) * g.Hh + w.h;
-        float M = -INFINITY;
-        if (valid) {
-          for (int t = 0; t < p.unit_split; ++t) M = fmaxf(M, ld_cg_f(p.lse_part + t * p.part_rows + prow));
-          M = fmaxf(M, lse_own);
-        }
-        const float Ms = M == -INFINITY ? 0.f : M;
-        float tot = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < D; c += 16) {
-          uint32_t o[16];
-          if (ntile > 0) tmem_ld16(tO + c, o);   // uniform over the warpgroup
-          if (valid) {
-            float acc[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-            for (int t = 0; t <= p.unit_split; ++t) {
-              const bool own = t == p.unit_split;
-              const float wt = expf((own ? lse_own : ld_cg_f(p.lse_part + t * p.part_rows + prow)) - Ms);
-              if (wt != 0.f) {
-                if (own) {
-#pragma unroll
-                  for (int j = 0; j < 16; ++j) acc[j] = fmaf(wt, __uint_as_float(o[j]) * inv, acc[j]);
-                } else {
-                  const float* src = p.o_part + (t * p.part_rows + prow) * D + c;
-#pragma unroll
-                  for (int j = 0; j < 4; ++j) {
-                    const float4 v = ld_cg_f4(src + 4 * j);
-                    acc[4 * j] = fmaf(wt, v.x, acc[4 * j]);
-                    acc[4 * j + 1] = fmaf(wt, v.y, acc[4 * j + 1]);
-                    acc[4 * j + 2] = fmaf(wt, v.z, acc[4 * j + 2]);
-                    acc[4 * j + 3] = fmaf(wt, v.w, acc[4 * j + 3]);
-                  }
-                }
-                if (c == 0) tot += wt;
-              }
-            }
-            const float it = tot > 0.f ? 1.f / tot : 0.f;
-            uint4* dst = reinterpret_cast<uint4*>(p.o_final + prow * D + c);
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              uint4 u;
-              u.x = pack_bf16x2(acc[8 * j + 0] * it, acc[8 * j + 1] * it);
-              u.y = pack_bf16x2(acc[8 * j + 2] * it, acc[8 * j + 3] * it);
-              u.z = pack_bf16x2(acc[8 * j + 4] * it, acc[8 * j + 5] * it);
-              u.w = pack_bf16x2(acc[8 * j + 6] * it, acc[8 * j + 7] * it);
-              dst[j] = u;
-            }
-          }
-        }
-        if (valid) {
-          const float lse = M == -INFINITY ? -INFINITY : Ms + logf(tot);
-          if (p.lse_final != nullptr) {
-            p.lse_final[prow] = lse;   // rows in the partials' order
-          } else if (p.lse != nullptr) {
-            // natural [B][H][S] order, as the fused forward writes it
-            const int64_t li = (static_cast<int64_t>(bv % p.lse_B) * p.lse_H + (bv / p.lse_B) * g.Hh + w.h) *
-                                   p.lse_S + gq;
-            p.lse[li] = lse;
-          }
-        }
-        continue;
-      }
       if (ntile > 0) {
         ok = mbar_wait(smem_addr(&sm.o_done[wg]), od_cnt & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
@@ -692,13 +602,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (merged) {
-        // First-phase unit of a merged ring launch: its partial rows are written;
-        // publish them to the query tile's tail unit (one count per warp).
-        chunk_stores_fence();
-        __syncwarp();
-        if (lane == 0) red_release_add(done, 1);
-      }
     }
   }
 
@@ -714,6 +617,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int per_half = p.pull_chunks / 2;
       const int64_t half = p.pull_block_bytes;
       const int64_t total = static_cast<int64_t>(g.NR - 1) * p.pull_chunks;
+      // The fetch streams every other block through L2 once: evict-first, so
+      // that it does not displace the key/value tiles the units are reusing
+      // (their TMA loads are evict-last).
+      const uint64_t pol = l2_policy_evict_first();
       for (int64_t c = cw; c < total; c += ncw) {
         if (abort_raised(ctl.wb)) break;
         const int jj = static_cast<int>(c / p.pull_chunks);
@@ -730,10 +637,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint4 r[kU];
 #pragma unroll
           for (int u = 0; u < kU; ++u)
-            if (i + u * 512 < n) r[u] = ld_stream_v4(src + i + u * 512);
+            if (i + u * 512 < n) r[u] = ld_stream_v4_policy(src + i + u * 512, pol);
 #pragma unroll
           for (int u = 0; u < kU; ++u)
-            if (i + u * 512 < n) st_v4(dst + i + u * 512, r[u]);
+            if (i + u * 512 < n) st_v4_policy(dst + i + u * 512, r[u], pol);
         }
         chunk_stores_fence();
         __syncwarp();
@@ -774,9 +681,7 @@ cudaError_t launch_impl(const FwdLaunch& L, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
-  // A merged ring launch is cooperative too: tail units wait for first-phase
-  // units of other CTAs.
-  cfg.numAttrs = (PARTIAL && (L.params.pull_chunks > 0 || L.params.merge_done != nullptr)) ? 1 : 0;
+  cfg.numAttrs = (PARTIAL && L.params.pull_chunks > 0) ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, L.tm_q, L.tm_k, L.tm_v, L.params);
 }
 

@@ -59,19 +59,6 @@ struct FwdParams {
   int64_t pull_block_bytes;
   int pull_chunk_bytes;
   int pull_chunks;
-  // Merged ring launch (partial mode with unit_steps): the units of the first
-  // phase (unit_t0 < unit_split) write their partials and then count, per warp,
-  // in merge_done[(b * Hh + h) * merge_tiles + query tile] (merge_tiles = 2 x
-  // query-tile pairs, so the second tile of a ragged pair has its own count); the tail unit of a
-  // query tile waits until its count reaches 4 * unit_split, merges those
-  // partials with its own on-chip state in the order of the merge kernel, and
-  // writes o_final (bf16, [row blocks from q_rb0][T][Hh][D]) and lse_final
-  // ([rows], partial-row order) or, with lse_final null, lse (natural order).
-  // merge_done null: the tail unit writes part unit_split like the others.
-  int* merge_done;
-  int merge_tiles;
-  __nv_bfloat16* o_final;
-  float* lse_final;
   int* status;                 // device status word (0 = ok)
   uint64_t wait_limit_ns;      // budget of one in-kernel wait
 };

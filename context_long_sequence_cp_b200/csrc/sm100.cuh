@@ -168,11 +168,6 @@ __device__ __forceinline__ void red_release_add(int* count, int v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(count), "r"(v) : "memory");
 }
 
-// Loads of data other CTAs of this kernel wrote (ordered after an acquire of
-// their release count): cached in L2 only, never in a possibly stale L1.
-__device__ __forceinline__ float4 ld_cg_f4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
-__device__ __forceinline__ float ld_cg_f(const float* p) { return __ldcg(p); }
-
 // 16-byte streaming load (read-only for the kernel's lifetime, no L1 allocation)
 // and store.
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
@@ -184,6 +179,21 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
 }
 __device__ __forceinline__ void st_v4(void* p, const uint4& v) {
   asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+// The same load and store with an L2 cache policy (createpolicy): a stream
+// marked evict-first passes through L2 without displacing what other loads
+// marked evict-last keep there.
+__device__ __forceinline__ uint4 ld_stream_v4_policy(const void* p, uint64_t policy) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(policy));
+  return v;
+}
+__device__ __forceinline__ void st_v4_policy(void* p, const uint4& v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w), "l"(policy)
                : "memory");
 }
 

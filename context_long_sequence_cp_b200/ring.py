@@ -11,15 +11,13 @@ bandwidth, so rank r fetches block (r + t) mod N straight from its owner rather
 than having it relayed hop by hop: the same bytes per rank (N - 1 blocks), no
 chain of per-step hand-offs. Each rank exposes its own block in a slot buffer
 the others map through CUDA IPC. The whole forward is ONE persistent,
-cooperative kernel launch: the first half of the ring
+cooperative kernel launch (``cp_attn_fwd_ring``): the first half of the ring
 steps runs step-major, one unit per (step, query-tile pair), starting on the
 rank's own block; then each pair walks the remaining steps in one unit. Two
 copy warps of every CTA meanwhile load the other blocks over NVLink, in ring
 order, into local slots, publishing per-block arrival counts that the units
-wait on; the tail unit of each query tile merges the first-phase partials
-of that tile on chip once they are written (``cp_attn_fwd_ring_merged``), so
-the launch returns the rank's rows of full attention. The transfer overlaps the
-math inside one kernel and needs no copy engine, stream or event between them (a device-to-device
+wait on. The transfer overlaps the math inside one
+kernel and needs no copy engine, stream or event between them (a device-to-device
 copy issued on another stream does not progress while the persistent kernel
 holds every SM). The ranks meet at ONE host barrier per call, after every rank's
 own block is in place. Slot buffers alternate between calls, so that a rank may
@@ -33,7 +31,7 @@ from typing import Callable, Optional, Sequence
 
 import torch
 
-from . import DeviceBuffer, PeerBuffer, Plan, _check, copy_async, lib
+from . import DeviceBuffer, PeerBuffer, Plan, _check, copy_async, lib, merge_partials
 
 SLOT_SETS = 2   # call c uses slot set c mod 2
 
@@ -87,8 +85,9 @@ class RingRank:
         self.slots = DeviceBuffer(SLOT_SETS * self.set_bytes)
         self.peer_bases: Optional[list] = None
         self.arrived = torch.zeros(N, dtype=torch.int32, device=self.device)
-        # the merged launch's first-phase partials and completion counts
-        self.workspace = torch.empty(plan.ring_merged_workspace_bytes(), dtype=torch.uint8, device=self.device)
+        P = plan.ring_parts()
+        self.o_parts = torch.empty(P, self.rows, D, dtype=torch.float32, device=self.device)
+        self.lse_parts = torch.empty(P, self.rows, dtype=torch.float32, device=self.device)
         self.calls = 0
         self.copy_stream = torch.cuda.Stream(device=self.device)
         self.fill_done = torch.cuda.Event()
@@ -138,32 +137,31 @@ class RingRank:
             copy_async(v_all + r * self.block_bytes, v.data_ptr(), self.block_bytes, cs)
             self.fill_done.record(cs)
 
-        o = torch.empty(self.shape, dtype=torch.bfloat16, device=self.device)
-        lse = torch.empty(self.rows, dtype=torch.float32, device=self.device)
-
         def launch():
             st.wait_event(self.fill_done)
             pk, pv = self.pull_sources(c) if N > 1 else (None, None)
-            _launch_ring(self.plan, r, q, k_all, v_all, pk, pv, self.arrived if N > 1 else None, o, lse,
-                         self.workspace, st)
+            _launch_ring(self.plan, r, q, k_all, v_all, pk, pv, self.arrived if N > 1 else None, self.o_parts,
+                         self.lse_parts, st)
 
         run_ring(fill, self.fill_done.synchronize, self.barrier, launch)
-        return o, lse
+        o, lse = merge_partials(self.o_parts, self.lse_parts, stream=st)
+        return o.view(self.shape), lse
 
     def close(self):
         self.slots.close()
 
 
-def _launch_ring(plan, rank, q, k_all, v_all, pk, pv, arrived, o, lse, workspace, st):
+def _launch_ring(plan, rank, q, k_all, v_all, pk, pv, arrived, o_parts, lse_parts, st):
     if pk is None:
         pka = pva = None
     else:
         pka = ctypes.cast((ctypes.c_void_p * len(pk))(*pk), ctypes.c_void_p)
         pva = ctypes.cast((ctypes.c_void_p * len(pv))(*pv), ctypes.c_void_p)
-    _check("cp_attn_fwd_ring_merged",
-           lib().cp_attn_fwd_ring_merged(plan.handle, rank, _vp(q.data_ptr()), _vp(k_all), _vp(v_all), pka, pva,
-                                         None if arrived is None else _vp(arrived.data_ptr()), _vp(o.data_ptr()),
-                                         _vp(lse.data_ptr()), _vp(workspace.data_ptr()), _vp(st.cuda_stream)))
+    _check("cp_attn_fwd_ring",
+           lib().cp_attn_fwd_ring(plan.handle, rank, _vp(q.data_ptr()), _vp(k_all), _vp(v_all), pka, pva,
+                                  None if arrived is None else _vp(arrived.data_ptr()), _vp(o_parts.data_ptr()),
+                                  _vp(lse_parts.data_ptr()),
+                                  _vp(st.cuda_stream)))
 
 
 def _vp(x: int):

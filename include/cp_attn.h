@@ -115,11 +115,6 @@ CP_API int64_t cp_attn_plan_tile_counts(cp_attn_plan_t plan, int64_t* per_rank);
 /* Number of work items (pairs of 128-row query tiles) in the plan's work list. */
 CP_API int64_t cp_attn_plan_num_items(cp_attn_plan_t plan);
 
-/* Units of the split forward of a short problem (see cp_attn_workspace_bytes),
- * 0 when the plan does not split; *split_steps (host, may be NULL) receives the
- * number of first-phase ring steps (0 when not split). Negative on error. */
-CP_API int64_t cp_attn_plan_split_units(cp_attn_plan_t plan, int* split_steps);
-
 /*
  * Static schedule of the attention kernel: one persistent CTA per SM runs a
  * contiguous run of the work list, assigned at plan time by giving each item,
@@ -133,14 +128,8 @@ CP_API int64_t cp_attn_plan_cta_loads(cp_attn_plan_t plan, int64_t* per_cta);
 
 /*
  * Workspace bytes needed by cp_attn_fwd (with_partials = 0) or
- * cp_attn_fwd_partials (with_partials = 1). 4 * B*S*H*D*2 bytes (Q, K, V and O
- * head groups) for Ulysses. For contiguous/zigzag plans 0, except for short
- * problems (fewer than 4 work items per SM, N >= 2): their fused forward splits
- * each work item's ring walk into units over ring steps, one per step before
- * split = ceil(N/2) (1 for N = 2) and one tail unit over the rest that merges
- * the others' partials on chip; the workspace holds those fp32 partials
- * (split x B*S*H x (D + 1) x 4 bytes) and per-query-tile completion counts.
- * cp_attn_fwd given no workspace for such a plan runs the unsplit launch.
+ * cp_attn_fwd_partials (with_partials = 1). 0 for contiguous/zigzag fused
+ * calls; 4 * B*S*H*D*2 bytes (Q, K, V and O head groups) for Ulysses.
  */
 CP_API size_t cp_attn_workspace_bytes(cp_attn_plan_t plan, int with_partials);
 
@@ -153,10 +142,8 @@ CP_API size_t cp_attn_workspace_bytes(cp_attn_plan_t plan, int with_partials);
  *   q, k, v : bf16, in the plan's layout (see above), device
  *   o       : bf16, same layout and size as q, device (written)
  *   lse     : float32 [B][H][S] natural token order, device (written); may be NULL
- *   workspace : device, cp_attn_workspace_bytes(plan, 0) bytes (NULL if 0; for a
- *             short contiguous/zigzag problem NULL selects the unsplit launch)
- * q, k, v must not overlap o or workspace. The split launch of a short problem
- * is cooperative (its tail units wait, bounded, for their first-phase units).
+ *   workspace : device, cp_attn_workspace_bytes(plan, 0) bytes (NULL if 0)
+ * q, k, v must not overlap o or workspace.
  */
 CP_API int cp_attn_fwd(cp_attn_plan_t plan, const void* q, const void* k, const void* v,
                 void* o, float* lse, void* workspace, cp_stream_t stream);
@@ -261,32 +248,6 @@ CP_API int cp_attn_fwd_ring(cp_attn_plan_t plan, int rank, const void* q, void* 
  * cp_attn_check; the context stays usable. */
 CP_API int cp_attn_fwd_ring_external(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all,
                                      int* arrived, float* o_parts, float* lse_parts, cp_stream_t stream);
-
-/* The rank's ring forward in one launch with its merge done on chip: the same
- * units, order and copy warps as cp_attn_fwd_ring, but the tail unit of each
- * query tile (ring steps [split, N)) waits, bounded, until the first-phase units
- * of that tile (steps 0 .. split - 1) have written their partials, merges them
- * with its own online-softmax state and writes the rank's rows of full
- * attention: no tail partial and no separate merge launch. The combination
- * follows cp_merge_partials' formula, order and arithmetic, so o and lse are
- * bit-identical to cp_attn_fwd_ring followed by cp_merge_partials. Page
- * "序列与上下文并行", section "上下文并行：注意力本身切分" (partials merged by online
- * softmax). For N <= 2 (no tail phase) the partials are merged by the merge
- * kernel after the launch.
- *   q, k_all, v_all, pull_k, pull_v, arrived : as cp_attn_fwd_ring
- *   o         : bf16 [B][S/N][H][D], the rank's rows (written), device
- *   lse       : float32 [B*(S/N)*H], natural log, rows as o (written), device
- *   workspace : cp_attn_ring_merged_workspace_bytes(plan) bytes, device,
- *               16-byte aligned (first-phase partials and completion counts;
- *               the counts are reset on `stream` before the launch)
- * The launch is cooperative (all CTAs resident), so every wait ends. Errors:
- * as cp_attn_fwd_ring; CP_ERR_INVALID_ARG for a NULL o, lse or workspace;
- * CP_ERR_ALIGNMENT for o or workspace not 16-byte or lse not 4-byte aligned.
- */
-CP_API size_t cp_attn_ring_merged_workspace_bytes(cp_attn_plan_t plan);
-CP_API int cp_attn_fwd_ring_merged(cp_attn_plan_t plan, int rank, const void* q, void* k_all, void* v_all,
-                                   const void* const* pull_k, const void* const* pull_v, int* arrived, void* o,
-                                   float* lse, void* workspace, cp_stream_t stream);
 
 /* Number of partials cp_attn_fwd_ring writes (N for N <= 3, else ceil(N/2) + 1),
  * or a negative status (CP_ERR_UNSUPPORTED for Ulysses). */

@@ -112,21 +112,9 @@ def test_workspace_and_map_sizes():
     assert p.index_map_len() == 8 * 2 * 16384
     assert p.tile_counts()[0] == [2 * 4 * 128 * 128] * 8
     z = cp.Plan(1, 16, 4096, 128, 4, True, "zigzag")
+    assert z.workspace_bytes(False) == 0 and z.workspace_bytes(True) == 0
     assert z.index_map_len() == 4096
     assert z.num_items() == 4 * 16 * 4     # ranks x heads x query-tile pairs (T=1024)
-    # 256 items < 4 per SM: the fused forward splits every walk into ring-step units,
-    # steps 0 and 1 one unit each, then a tail over steps 2-3 (3 units per item)
-    assert z.split_units() == (3 * 256, 2)
-    up = lambda x: -(-x // 256) * 256
-    rows = 4096 * 16
-    assert z.workspace_bytes(False) == up(2 * rows * 128 * 4) + up(2 * rows * 4) + up(4 * 16 * 2 * 4 * 4)
-    assert z.workspace_bytes(True) == 0
-    big = cp.Plan(1, 32, 32768, 128, 8, True, "zigzag")        # 2048 items: not split
-    assert big.split_units() == (0, 0) and big.workspace_bytes(False) == 0
-    two = cp.Plan(1, 2, 1024, 64, 2, True, "zigzag")            # N = 2: step 0, then a tail over step 1
-    assert two.split_units() == (2 * 2 * 2 * 2, 1)
-    one = cp.Plan(1, 2, 700, 128, 1, True, "contiguous")        # one rank: nothing to split
-    assert one.split_units() == (0, 0) and one.workspace_bytes(False) == 0
 
 
 def _executed_key_tiles(S, N, layout, causal, tile=128):

@@ -132,33 +132,3 @@ def _spiked_qkv(B, H, S, D, seed):
 def test_growing_row_max_rescales(layout, causal, D):
     q, k, v = _spiked_qkv(1, 2, 2048, D, 21)
     run_and_compare(q, k, v, 2, layout, causal, what=f"spiked {layout} causal={causal} D={D}")
-
-
-@pytest.mark.parametrize("B,H,S,D,N,layout,causal,seed", [
-    (1, 16, 4096, 128, 4, "zigzag", True, 1),        # the 4k workload's shape
-    (2, 3, 1024, 64, 2, "zigzag", True, 11),
-    (1, 2, 1000, 64, 5, "zigzag", True, 14),         # ragged chunks, 3 first-phase steps
-    (2, 2, 600, 128, 3, "contiguous", False, 15),    # ragged non-causal
-])
-def test_split_forward_matches_unsplit_launch(B, H, S, D, N, layout, causal, seed):
-    """A short problem's split forward (ring-step units merged on chip) against the
-    unsplit launch of the same plan (no workspace) and against the oracle."""
-    import ctypes
-    q, k, v = make_small(B, H, S, D, seed)
-    plan = cp.Plan(B, H, S, D, N, causal, layout)
-    assert plan.split_units()[0] > 0
-    qd, kd, vd = (G.to_layout(x, N, layout).cuda() for x in (q, k, v))
-    o_s, l_s = cp.attn_fwd(plan, qd, kd, vd)                  # the binding passes the workspace
-    o_u, l_u = torch.empty_like(qd), torch.empty(B, H, S, dtype=torch.float32, device="cuda")
-    rc = cp.lib().cp_attn_fwd(plan.handle, cp._ptr(qd), cp._ptr(kd), cp._ptr(vd), cp._ptr(o_u), cp._ptr(l_u), None,
-                              cp._stream(None))
-    assert rc == 0 and cp.check(plan) == 0
-    d = (o_s.float() - o_u.float()).abs()
-    assert d.max().item() <= G.TOL_O_MAX and d.mean().item() <= 1e-3
-    assert (l_s - l_u).abs().max().item() <= G.TOL_LSE
-    bb, hh, ii = np.meshgrid(np.arange(B), np.arange(H), np.arange(S), indexing="ij")
-    rows = np.stack([bb.ravel(), hh.ravel(), ii.ravel()], 1).astype(np.int64)
-    o_gpu = G.gather_rows(o_s, B, S, H, N, layout, rows)
-    lse_gpu = l_s.cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]].astype(np.float64)
-    o_ref, lse_ref = G.oracle_rows(q, k, v, rows, causal)
-    G.assert_within(G.errors(o_gpu, o_ref, lse_gpu, lse_ref), "split forward")

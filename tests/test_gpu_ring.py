@@ -260,44 +260,3 @@ def test_ring_rank_full_size_sampled_rows(name, layout, rank):
     d = np.abs(got - o_ref)
     assert d.max() <= G.TOL_O_MAX and d.mean() <= G.TOL_O_MEAN, d.max()
     assert np.abs(got_l - l_ref).max() <= G.TOL_LSE
-
-
-@pytest.mark.parametrize("B,H,S,D,N,layout,causal,pull", [
-    (1, 2, 1024, 128, 4, "zigzag", True, True),
-    (2, 2, 1536, 64, 3, "contiguous", True, False),
-    (1, 3, 1920, 128, 5, "zigzag", True, True),       # ragged query-tile pair
-    (1, 2, 4096, 128, 8, "zigzag", True, True),
-    (1, 2, 2048, 128, 8, "contiguous", False, False),
-    (1, 2, 512, 64, 2, "contiguous", False, True),     # no tail phase: launch, then the merge kernel
-])
-def test_merged_ring_launch_equals_launch_then_merge(B, H, S, D, N, layout, causal, pull):
-    """The on-chip merge of the tail units gives exactly the partials + merge kernel result."""
-    q, k, v = make_small(B, H, S, D, 120 + N)
-    plan = cp.Plan(B, H, S, D, N, causal, layout)
-    qd, kd, vd = (G.to_layout(x, N, layout).cuda() for x in (q, k, v))
-    f = lambda t: t.float().numpy()
-    o_ref_all, l_ref_all = A.attention(f(q), f(k), f(v), causal=causal)
-    pos = L.chunk_positions(S, N, layout)
-    ws = torch.empty(plan.ring_merged_workspace_bytes(), dtype=torch.uint8, device="cuda")
-    for r in range(N):
-        op, lp = cp.attn_fwd_ring(plan, r, qd[r], kd, vd)
-        o_u, l_u = cp.merge_partials(op, lp)
-        if pull:
-            ks, vs = torch.zeros_like(kd), torch.zeros_like(vd)
-            ks[r].copy_(kd[r])
-            vs[r].copy_(vd[r])
-            arrived = torch.zeros(N, dtype=torch.int32, device="cuda")
-            srcs = ([kd[j].data_ptr() for j in range(N)], [vd[j].data_ptr() for j in range(N)])
-            o_m, l_m = cp.attn_fwd_ring_merged(plan, r, qd[r], ks, vs, srcs[0], srcs[1], arrived, workspace=ws)
-        else:
-            o_m, l_m = cp.attn_fwd_ring_merged(plan, r, qd[r], kd, vd, workspace=ws)
-        assert cp.check(plan) == 0
-        assert torch.equal(o_m.reshape(-1).view(torch.int16), o_u.reshape(-1).view(torch.int16)), r
-        assert torch.equal(l_m.view(torch.int32), l_u.view(torch.int32)), r
-        # and the rank's rows against the oracle
-        T = S // N
-        o_np = o_m.double().cpu().numpy().reshape(B, T, H, D)
-        d = np.abs(o_np - o_ref_all[:, pos[r]])
-        assert d.max() <= G.TOL_O_MAX and d.mean() <= G.TOL_O_MEAN, (r, d.max())
-        l_np = l_m.double().cpu().numpy().reshape(B, T, H)
-        assert np.abs(l_np - l_ref_all[:, :, pos[r]].transpose(0, 2, 1)).max() <= G.TOL_LSE
