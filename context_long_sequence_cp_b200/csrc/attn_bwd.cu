@@ -59,24 +59,6 @@ constexpr int kWarpMma = 8;
 constexpr int kWarpTma = 9;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Column pairs (bit j of each 32-column run: columns 2j, 2j + 1) of a whole tile
-// whose exponentials run on the FMA pipe (exp2_poly_x2) instead of the MUFU: in
-// the P phase both warpgroups exponentiate the same tile at once, so the MUFU is
-// the busy pipe while the FMA pipe idles.
-#ifndef CP_BWD_POLY_PAIRS
-#define CP_BWD_POLY_PAIRS 0x0u
-#endif
-constexpr uint32_t kBwdPolyPairs = CP_BWD_POLY_PAIRS;
-
-__device__ __forceinline__ void exp2_pair(bool poly, float x0, float x1, float& e0, float& e1) {
-  if (poly) {
-    exp2_poly_x2(x0, x1, e0, e1);
-  } else {
-    e0 = ex2_approx(x0);
-    e1 = ex2_approx(x1);
-  }
-}
-
 template <int D>
 struct BwdCfg {
   static constexpr int kTileBytes = kTile * D * 2;   // one 128 x D bf16 tile
@@ -508,12 +490,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               float x0, x1, x2, x3;
               f2_unpack(f2_fma(f2_pack(__uint_as_float(sa[2 * j]), __uint_as_float(sa[2 * j + 1])), sl2_2, na), x0, x1);
               f2_unpack(f2_fma(f2_pack(__uint_as_float(sb[2 * j]), __uint_as_float(sb[2 * j + 1])), sl2_2, nb), x2, x3);
-              const bool poly = (kBwdPolyPairs >> j) & 1u;
-              float e0, e1, e2, e3;
-              exp2_pair(poly, x0, x1, e0, e1);
-              exp2_pair(poly, x2, x3, e2, e3);
-              pk[j] = pack_bf16x2(e0, e1);
-              pk[16 + j] = pack_bf16x2(e2, e3);
+              pk[j] = pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+              pk[16 + j] = pack_bf16x2(ex2_approx(x2), ex2_approx(x3));
             }
           } else {
 #pragma unroll
@@ -830,9 +808,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         x0, x1);
               const uint64_t g2 =
                   f2_sub(f2_pack(__uint_as_float(da[cc][2 * j]), __uint_as_float(da[cc][2 * j + 1])), dr_2);
-              float e0, e1;
-              exp2_pair((kBwdPolyPairs >> j) & 1u, x0, x1, e0, e1);
-              f2_unpack(f2_mul(f2_pack(e0, e1), g2), d0, d1);
+              f2_unpack(f2_mul(f2_pack(ex2_approx(x0), ex2_approx(x1)), g2), d0, d1);
               dk[cc][j] = pack_bf16x2(d0, d1);
             }
         } else {

@@ -489,11 +489,6 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   return r;
 }
 
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
 __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
@@ -508,36 +503,6 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
-}
-
-// 2^x for a pair of floats on the FMA pipe instead of the MUFU (two lanes per
-// packed instruction), for finite x <= 2^22 (inputs below -125 give 2^-125).
-// Range reduction after Cody and Waite (Software Manual for the Elementary
-// Functions, 1980): adding 1.5 * 2^23 rounds x to the nearest integer n, held in
-// the low mantissa bits of the sum, and f = x - n lies in [-1/2, 1/2]. 2^f is a
-// degree-3 polynomial whose coefficients are the relative-error minimax fit on
-// [-1/2, 1/2] (Remez exchange, fp64, rounded to fp32): relative error 7.5e-5,
-// well under the 2^-9 of the bf16 rounding P goes through. 2^n is applied by
-// adding n << 23 to the polynomial's bits: (bits(x + 1.5 * 2^23) << 23) is
-// n << 23 modulo 2^32, because the constant's own bits vanish in the shift.
-constexpr float kExp2C0 = 0.99992805719375610f;
-constexpr float kExp2C1 = 0.69326096773147583f;
-constexpr float kExp2C2 = 0.24261112511157990f;
-constexpr float kExp2C3 = 0.05517166852951050f;
-
-__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, float& y1) {
-  const uint64_t round = f2_pack(12582912.0f, 12582912.0f);
-  const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t t = f2_add(x, round);
-  const uint64_t f = f2_sub(x, f2_sub(t, round));
-  uint64_t p = f2_fma(f, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
-  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
-  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
-  float tl, th, pl, ph;
-  f2_unpack(t, tl, th);
-  f2_unpack(p, pl, ph);
-  y0 = __uint_as_float(__float_as_uint(pl) + (__float_as_uint(tl) << 23));
-  y1 = __uint_as_float(__float_as_uint(ph) + (__float_as_uint(th) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
