@@ -188,16 +188,49 @@ int assign_greedy(std::vector<WorkItem>& items, const std::vector<int64_t>& cost
   return n_cta;
 }
 
-void schedule_items(cp_attn_plan_s* p, int n_cta) {
-  const int n = static_cast<int>(p->items.size());
-  std::vector<int64_t> cost(n);
+// Assigns the items (already in the grouped order: items that share keys/values
+// next to each other) twice: in that order and longest-first over the whole list.
+// The grouped assignment is kept unless longest-first lowers the modelled finish
+// time of the last CTA by more than 2%: grouping keeps the K/V of the items that
+// run together shared in L2, which only balance on few items per CTA (short
+// sequences, whose K/V fits in L2 anyway) should override.
+template <class CostOf>
+int assign_balanced(std::vector<WorkItem>& items, CostOf cost_of, int n_cta, std::vector<int>& cta_begin,
+                    std::vector<int64_t>& cta_load) {
+  const int n = static_cast<int>(items.size());
+  std::vector<WorkItem> lpt = items;
+  std::vector<int64_t> cost(n), cost_lpt(n);
+  for (int i = 0; i < n; ++i) cost[i] = cost_of(items[i]);
+  std::vector<int> order(n);
+  for (int i = 0; i < n; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
   for (int i = 0; i < n; ++i) {
-    const WorkItem& w = p->items[i];
+    lpt[i] = items[order[i]];
+    cost_lpt[i] = cost[order[i]];
+  }
+  std::vector<int> begin_lpt;
+  std::vector<int64_t> load_lpt;
+  const int n_grouped = assign_greedy(items, cost, n_cta, cta_begin, cta_load);
+  const int n_lpt = assign_greedy(lpt, cost_lpt, n_cta, begin_lpt, load_lpt);
+  int64_t max_grouped = 0, max_lpt = 0;
+  for (int64_t l : cta_load) max_grouped = l > max_grouped ? l : max_grouped;
+  for (int64_t l : load_lpt) max_lpt = l > max_lpt ? l : max_lpt;
+  if (max_lpt * 100 < max_grouped * 98) {
+    items.swap(lpt);
+    cta_begin.swap(begin_lpt);
+    cta_load.swap(load_lpt);
+    return n_lpt;
+  }
+  return n_grouped;
+}
+
+void schedule_items(cp_attn_plan_s* p, int n_cta) {
+  auto cost_of = [p](const WorkItem& w) {
     const int rq = w.rb / p->g.B;
     const int* off = p->step_off.data() + static_cast<size_t>(rq * p->npairs + w.qp) * (p->g.NR + 1);
-    cost[i] = 2 * static_cast<int64_t>(off[p->g.NR] - off[0]) + kItemOverheadHalfTiles;
-  }
-  p->n_cta = assign_greedy(p->items, cost, n_cta, p->cta_begin, p->cta_load);
+    return 2 * static_cast<int64_t>(off[p->g.NR] - off[0]) + kItemOverheadHalfTiles;
+  };
+  p->n_cta = assign_balanced(p->items, cost_of, n_cta, p->cta_begin, p->cta_load);
 }
 
 // Walks and schedules of the two backward kernels. A walk entry's class is
@@ -243,9 +276,8 @@ void build_bwd(cp_attn_plan_s* p, int n_cta) {
       if (x.h / 2 != y.h / 2) return x.h / 2 < y.h / 2;
       return x.cost > y.cost;
     });
-    std::vector<int64_t> cost(b.items.size());
-    for (size_t i = 0; i < b.items.size(); ++i) cost[i] = 2 * static_cast<int64_t>(b.items[i].cost) + kItemOverheadHalfTiles;
-    b.n_cta = assign_greedy(b.items, cost, n_cta, b.cta_begin, b.cta_load);
+    auto cost_of = [](const WorkItem& w) { return 2 * static_cast<int64_t>(w.cost) + kItemOverheadHalfTiles; };
+    b.n_cta = assign_balanced(b.items, cost_of, n_cta, b.cta_begin, b.cta_load);
   }
 }
 

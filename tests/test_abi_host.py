@@ -150,6 +150,20 @@ def test_static_schedule_is_balanced_and_complete(layout):
     assert loads.sum() == 2 * walked + 3 * p.num_items()
 
 
+def test_static_schedule_few_items_per_cta_is_longest_first():
+    # zigzag_4k: 256 items on 148 CTAs. Grouping items by head pair would leave the
+    # late groups' long items on CTAs already holding short ones (modelled max/mean
+    # 1.59); the longest-first assignment ends at the largest single item.
+    w = WORKLOADS["zigzag_4k"]
+    p = cp.Plan(w.B, w.H, w.S, w.D, w.N, True, "zigzag")
+    loads = np.array(p.cta_loads())
+    walked = _executed_key_tiles(w.S, w.N, "zigzag", True) * w.H
+    assert loads.sum() == 2 * walked + 3 * p.num_items()
+    largest_item = 2 * (w.S // 128) + 3          # the last pair walks every key tile
+    assert loads.max() == largest_item
+    assert loads.max() / loads.mean() < 1.05
+
+
 def test_static_schedule_small_plan_one_item_per_cta():
     p = cp.Plan(1, 2, 256, 64, 4, False, "contiguous")   # 4 ranks x 2 heads x 1 pair
     loads = p.cta_loads()
