@@ -26,7 +26,10 @@
 //                      [128,256), dQ [256,256+D), dS double-buffered as bf16 in
 //                      [384,448) and [448,512); dS (from TMEM) times K (MN-major)
 //                      accumulates dQ. S and dP of the next key tile are computed
-//                      while the current dS is formed.
+//                      while the current dS is formed. K and V come through
+//                      rings of their own: V is released once dP has read it, K
+//                      (3 stages at D = 128) only once dQ has, so the next tiles'
+//                      loads are in flight while a tile's dS is formed.
 // The dK/dV and dQ kernels recompute S and dP each (7 tile products per tile
 // pair instead of 5 with an atomic dQ): the price of having no atomics.
 //
@@ -65,6 +68,10 @@ struct BwdCfg {
   static constexpr int kBlocks = D / 64;             // 128-byte column blocks
   static constexpr int kBlockBytes = kTile * 128;    // 16 KB
   static constexpr int kStages = D == 128 ? 2 : 4;
+  // dQ kernel: K is held from S(e) until dQ(e) has read it, V only until dP(e)
+  // has, so the two have rings of their own and K the deeper one.
+  static constexpr int kKStages = D == 128 ? 3 : 5;
+  static constexpr int kVStages = D == 128 ? 2 : 4;
   static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);   // both operands K-major
   static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, 0, 1);   // A from TMEM, B MN-major
 };
@@ -220,10 +227,11 @@ template <int D>
 struct alignas(1024) QSmem {
   __nv_bfloat16 q[kTile * D];
   __nv_bfloat16 dout[kTile * D];
-  __nv_bfloat16 k[BwdCfg<D>::kStages][kTile * D];
-  __nv_bfloat16 v[BwdCfg<D>::kStages][kTile * D];
+  __nv_bfloat16 k[BwdCfg<D>::kKStages][kTile * D];
+  __nv_bfloat16 v[BwdCfg<D>::kVStages][kTile * D];
   uint64_t q_full, q_empty;
-  uint64_t kv_full[BwdCfg<D>::kStages], kv_empty[BwdCfg<D>::kStages];
+  uint64_t k_full[BwdCfg<D>::kKStages], k_empty[BwdCfg<D>::kKStages];
+  uint64_t v_full[BwdCfg<D>::kVStages], v_empty[BwdCfg<D>::kVStages];
   uint64_t s_full;
   uint64_t sdp_free;   // both warpgroups have read S and dP of the current tile
   uint64_t p_full[2];
@@ -598,9 +606,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(smem_addr(&sm.q_full), 1);
     mbar_init(smem_addr(&sm.q_empty), 1);
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(smem_addr(&sm.kv_full[s]), 1);
-      mbar_init(smem_addr(&sm.kv_empty[s]), 1);
+    for (int s = 0; s < C::kKStages; ++s) {
+      mbar_init(smem_addr(&sm.k_full[s]), 1);
+      mbar_init(smem_addr(&sm.k_empty[s]), 1);
+    }
+    for (int s = 0; s < C::kVStages; ++s) {
+      mbar_init(smem_addr(&sm.v_full[s]), 1);
+      mbar_init(smem_addr(&sm.v_empty[s]), 1);
     }
     mbar_init(smem_addr(&sm.s_full), 1);
     mbar_init(smem_addr(&sm.sdp_free), 256);
@@ -632,7 +644,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ------------------------------------------------------------ TMA producer
     const uint64_t pol_q = l2_policy_evict_first();
     const uint64_t pol_kv = l2_policy_evict_last();
-    int q_iter = 0, kv_idx = 0;
+    int q_iter = 0, k_idx = 0, v_idx = 0;
     bool ok = true;
     for (int it = __ldg(p.cta_begin + blockIdx.x); it < it_end && ok; ++it) {
       const WorkItem w = p.items[it];
@@ -655,24 +667,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t ent = __ldg(p.entries + e);
         const int rbk = entry_rank(ent) * g.B + bv;
         const int k0 = entry_tile(ent) * kTile;
-        const int st = kv_idx % C::kStages;
-        const int round = kv_idx / C::kStages;
-        if (round > 0) ok = mbar_wait(smem_addr(&sm.kv_empty[st]), (round - 1) & 1, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        const uint32_t bar = smem_addr(&sm.kv_full[st]);
-        mbar_arrive_expect_tx_elect(bar, 2 * C::kTileBytes);
-        for (int blk = 0; blk < C::kBlocks; ++blk) {
-          tma_load_4d_elect(smem_addr(sm.k[st]) + blk * C::kBlockBytes, &tm_k, bar, blk * 64, w.h, k0, rbk, pol_kv);
-          tma_load_4d_elect(smem_addr(sm.v[st]) + blk * C::kBlockBytes, &tm_v, bar, blk * 64, w.h, k0, rbk, pol_kv);
+        // K(e) into its ring, then V(e) into its own.
+        {
+          const int st = k_idx % C::kKStages;
+          const int round = k_idx / C::kKStages;
+          if (round > 0) ok = mbar_wait(smem_addr(&sm.k_empty[st]), (round - 1) & 1, ctl);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          const uint32_t bar = smem_addr(&sm.k_full[st]);
+          mbar_arrive_expect_tx_elect(bar, C::kTileBytes);
+          for (int blk = 0; blk < C::kBlocks; ++blk)
+            tma_load_4d_elect(smem_addr(sm.k[st]) + blk * C::kBlockBytes, &tm_k, bar, blk * 64, w.h, k0, rbk, pol_kv);
+          ++k_idx;
         }
-        ++kv_idx;
+        {
+          const int st = v_idx % C::kVStages;
+          const int round = v_idx / C::kVStages;
+          if (round > 0) ok = mbar_wait(smem_addr(&sm.v_empty[st]), (round - 1) & 1, ctl);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          const uint32_t bar = smem_addr(&sm.v_full[st]);
+          mbar_arrive_expect_tx_elect(bar, C::kTileBytes);
+          for (int blk = 0; blk < C::kBlocks; ++blk)
+            tma_load_4d_elect(smem_addr(sm.v[st]) + blk * C::kBlockBytes, &tm_v, bar, blk * 64, w.h, k0, rbk, pol_kv);
+          ++v_idx;
+        }
       }
     }
     if (!ok) {
+      // Abort: let every load this thread issued land before the CTA exits.
       const uint64_t lim = p.wait_limit_ns;
-      for (int idx = kv_idx - C::kStages; idx < kv_idx; ++idx)
-        if (idx >= 0) mbar_wait_drain(smem_addr(&sm.kv_full[idx % C::kStages]), (idx / C::kStages) & 1, lim);
+      for (int idx = k_idx - C::kKStages; idx < k_idx; ++idx)
+        if (idx >= 0) mbar_wait_drain(smem_addr(&sm.k_full[idx % C::kKStages]), (idx / C::kKStages) & 1, lim);
+      for (int idx = v_idx - C::kVStages; idx < v_idx; ++idx)
+        if (idx >= 0) mbar_wait_drain(smem_addr(&sm.v_full[idx % C::kVStages]), (idx / C::kVStages) & 1, lim);
       if (q_iter > 0) mbar_wait_drain(smem_addr(&sm.q_full), (q_iter - 1) & 1, lim);
     }
   } else if (warp == kWarpMma) {
@@ -700,8 +728,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int prev_st = 0;
       for (int e = e_begin; e < e_end; ++e) {
         const int nt = e - e_begin;
-        const int st = kv_idx % C::kStages;
-        ok = mbar_wait(smem_addr(&sm.kv_full[st]), (kv_idx / C::kStages) & 1, ctl);
+        const int st = kv_idx % C::kKStages;
+        const int vst = kv_idx % C::kVStages;
+        ok = mbar_wait(smem_addr(&sm.k_full[st]), (kv_idx / C::kKStages) & 1, ctl);
+        if (ok) ok = mbar_wait(smem_addr(&sm.v_full[vst]), (kv_idx / C::kVStages) & 1, ctl);
         // S and dP of the previous tile (of this or the previous item) are read.
         if (ok && tiles > 0) ok = mbar_wait(smem_addr(&sm.sdp_free), f_cnt & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
@@ -711,7 +741,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ++tiles;
         tc_fence_after();
         issue_nt<D>(tS, q_addr, smem_addr(sm.k[st]));      // S = Q K^T
-        issue_nt<D>(tP2, do_addr, smem_addr(sm.v[st]));    // dP = dO V^T
+        issue_nt<D>(tP2, do_addr, smem_addr(sm.v[vst]));   // dP = dO V^T
+        umma_commit_elect(smem_addr(&sm.v_empty[vst]));     // V is read by dP only
         issued = true;
         if (nt > 0) {
           // dS(e-1) of both warpgroups; waited before s_full(e) is committed, so
@@ -725,7 +756,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           umma_commit_elect(smem_addr(&sm.s_full));
           issue_dq<D>(tdQ, tdS + ((nt - 1) & 1) * 64, smem_addr(sm.k[prev_st]), acc);
           acc = true;
-          umma_commit_elect(smem_addr(&sm.kv_empty[prev_st]));
+          umma_commit_elect(smem_addr(&sm.k_empty[prev_st]));
         } else {
           umma_commit_elect(smem_addr(&sm.s_full));
         }
@@ -740,7 +771,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ++p_cnt;
         tc_fence_after();
         issue_dq<D>(tdQ, tdS + ((e_end - e_begin - 1) & 1) * 64, smem_addr(sm.k[prev_st]), acc);
-        umma_commit_elect(smem_addr(&sm.kv_empty[prev_st]));
+        umma_commit_elect(smem_addr(&sm.k_empty[prev_st]));
         umma_commit_elect(smem_addr(&sm.acc_done));
       }
       umma_commit_elect(smem_addr(&sm.q_empty));
