@@ -17,10 +17,13 @@
 //   warps 4-7  softmax warpgroup 1: query tile 1 of the item
 //   warp  8    allocates TMEM; lane 0 issues every tcgen05.mma
 //   warp  9    lane 0 issues every TMA load
-//   warps 10-11 idle
+//   warps 10-11 idle, except in a ring launch with a fused fetch, where they
+//              copy the other ranks' key/value blocks into local slots
 // TMEM (512 columns x 128 lanes): S0 [0,128) S1 [128,256) O0 [256,256+D)
-// O1 [256+D, 256+2D). P (bf16, packed 2 per column) overwrites the first 64
-// columns of its S tile and feeds the PV product straight from TMEM.
+// O1 [256+D, 256+2D). P (bf16, packed 2 per column) overwrites the upper 64
+// columns of its S tile (the scores of keys 64-127, in registers by then), so the
+// scores of keys 0-63 stay in TMEM for the rare recompute after a rescale, and
+// feeds the PV product straight from TMEM.
 // Shared memory: Q0, Q1 and a ring of NS key/value stages, each a 128 x D bf16
 // tile stored as D/64 column blocks of 128 rows x 128 B with the 128-byte swizzle
 // that TMA writes and the UMMA descriptors read.
