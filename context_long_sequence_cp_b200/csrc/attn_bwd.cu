@@ -709,6 +709,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // S(e-1), dP(e-1) (sdp_free); then dQ += dS(e-1) K(e-1) once dS(e-1) is in
     // its buffer (p_full). dS is double-buffered in TMEM columns [384, 512), so
     // the tensor core computes the next scores while the current dS is formed.
+    // V(e)'s stage is released once dP(e) has read it (its commit follows dP),
+    // K(e)'s once dQ(e) has.
     const uint32_t tS = tbase, tP2 = tbase + 128, tdQ = tbase + 256, tdS = tbase + 384;
     const uint32_t q_addr = smem_addr(sm.q), do_addr = smem_addr(sm.dout);
     int q_iter = 0, kv_idx = 0, p_cnt = 0, f_cnt = 0;
