@@ -83,6 +83,22 @@ def test_plan_argument_validation():
     assert cp.lib().cp_attn_plan_destroy(None) == 0
 
 
+def test_plan_size_limits():
+    """Shapes beyond what the kernels index are refused up front, before any table
+    is built: the packed walk entries (key rank < 2^12, key tile < 2^13), the
+    view's row blocks (B * N <= 2^20) and the element count (<= 2^40)."""
+    C = cp.CONTIGUOUS
+    assert _plan_status(1, 0, 256, 64, 4, 0, C, 0.0) == -1                # H <= 0
+    assert _plan_status(1, 2, 0, 64, 4, 0, C, 0.0) == -1                  # S <= 0
+    assert _plan_status(1, 2, 256, 64, 4, 0, C, float("nan")) == -1       # scale NaN
+    assert _plan_status(1, 2, 256, 64, 4, 0, C, float("inf")) == -1       # scale inf
+    assert _plan_status(1, 1, 4096, 64, 4096, 0, C, 0.0) == -2            # N = 2^12 ranks
+    assert _plan_status(1, 1, 8192 * 128, 64, 1, 0, C, 0.0) == -2         # 2^13 key tiles
+    assert _plan_status(1 << 18, 1, 8, 64, 8, 0, C, 0.0) == -2            # B * N = 2^21
+    assert _plan_status(1024, 1024, 1 << 16, 128, 1, 0, C, 0.0) == -2     # 2^43 elements
+    assert _plan_status(1, 2, 256, 64, 4, 0, C, 0.5) == 0                 # explicit scale
+
+
 @pytest.mark.parametrize("S,N,layout,causal", [
     (32768, 8, "zigzag", True), (32768, 8, "contiguous", True), (4096, 4, "zigzag", True),
     (131072, 4, "zigzag", True), (131072, 4, "contiguous", True), (256, 4, "contiguous", False),
