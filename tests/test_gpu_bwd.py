@@ -49,6 +49,8 @@ SMALL = [
     (2, 3, 384, 128, 3, "zigzag", True, 12),     # 64-token zigzag chunks: tiles straddle chunks
     (1, 2, 800, 128, 4, "contiguous", True, 13),  # ragged tails: 200 tokens per rank
     (1, 4, 2048, 128, 4, "zigzag", True, 14),
+    (1, 2, 3000, 64, 5, "zigzag", True, 15),     # D = 64, ragged 300-token chunks, walks past every ring
+    (2, 2, 1400, 128, 2, "contiguous", False, 16),  # ragged non-causal: 700 tokens per rank
 ]
 
 
