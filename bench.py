@@ -492,7 +492,7 @@ def ring_components(cp, torch, plan, w, dev, stream, legs, qz, kz, vz, oz, att_m
         ring_err = (r_o.float() - oz[0].float()).abs().max().item()
         if cp.check(plan) != 0 or not ring_err <= 2e-2:
             raise RuntimeError(f"ring rank 0 disagrees with the fused forward: {ring_err}")
-    ring_ms, c = legs.flushed(lambda: rr.forward(q0, kz[0], vz[0], stream), 7)
+    ring_ms, c = legs.flushed(lambda: rr.forward(q0, kz[0], vz[0], stream), 15)
     op_r, lp_r = rr.o_parts, rr.lse_parts
 
     def launch_only():
@@ -507,14 +507,14 @@ def ring_components(cp, torch, plan, w, dev, stream, legs, qz, kz, vz, oz, att_m
             cp.attn_fwd_ring_step(plan, 0, t, q0, kz[t], vz[t], op_s[t], lp_s[t], stream)
         cp.merge_partials(op_s, lp_s, o_out=ro, lse_out=rl)
 
-    ring_launch_ms, _ = legs.flushed(launch_only, 7)
-    ring_steps_ms, _ = legs.flushed(step_launches, 7)
+    ring_launch_ms, _ = legs.flushed(launch_only, 15)
+    ring_steps_ms, _ = legs.flushed(step_launches, 15)
     # The fused launch under the ring calls' own protocol (each call after an L2
     # flush, short enough to run at burst clocks), so that the share compares like
     # with like; the back-to-back figure of the attention leg runs under the power
     # cap and would flatter the ring.
     lse_f = torch.empty(w.B, w.H, w.S, dtype=torch.float32, device=dev)
-    fused_ms, fused_clock = legs.flushed(lambda: cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=lse_f), 5)
+    fused_ms, fused_clock = legs.flushed(lambda: cp.attn_fwd(plan, qz, kz, vz, o=oz, lse=lse_f), 7)
     if cp.check(plan) != 0:
         raise RuntimeError("ring runs failed")
     rr.close()
