@@ -39,12 +39,6 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
-               "r"(bytes)
-               : "memory");
-}
-
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -169,21 +163,8 @@ __device__ __forceinline__ void red_release_add(int* count, int v) {
 }
 
 // 16-byte streaming load (read-only for the kernel's lifetime, no L1 allocation)
-// and store.
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-__device__ __forceinline__ void st_v4(void* p, const uint4& v) {
-  asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-// The same load and store with an L2 cache policy (createpolicy): a stream
-// marked evict-first passes through L2 without displacing what other loads
-// marked evict-last keep there.
+// and store, with an L2 cache policy (createpolicy): a stream marked evict-first
+// passes through L2 without displacing what other loads marked evict-last keep.
 __device__ __forceinline__ uint4 ld_stream_v4_policy(const void* p, uint64_t policy) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
@@ -197,6 +178,8 @@ __device__ __forceinline__ void st_v4_policy(void* p, const uint4& v, uint64_t p
                : "memory");
 }
 
+// Arrive on an mbarrier and announce the transaction bytes the TMA copies of this
+// phase will bring; one elected lane of a converged warp.
 __device__ __forceinline__ void mbar_arrive_expect_tx_elect(uint32_t bar, uint32_t bytes) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -208,18 +191,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_elect(uint32_t bar, uint32
 
 // ---------------------------------------------------------------- TMA
 // 4-D tiled bulk tensor load global -> shared, completion signalled on an
-// mbarrier as transaction bytes. No multicast: the source is always this GPU.
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int c0, int c1, int c2, int c3, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar),
-      "l"(policy)
-      : "memory");
-}
-
-// The same load issued by one elected lane of a converged warp.
+// mbarrier as transaction bytes; issued by one elected lane of a converged warp.
+// No multicast: the source is always this GPU.
 __device__ __forceinline__ void tma_load_4d_elect(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                                   int c0, int c1, int c2, int c3, uint64_t policy) {
   asm volatile(
@@ -281,38 +254,12 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 in, fp32 accumulate).
-__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                        uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16.
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                        uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive (once) on an mbarrier when all previously issued tcgen05 ops of this thread complete.
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100 version 1.
-//   addr: byte address in shared memory; lbo/sbo: byte offsets (multiples of 16).
-// Forms issued by one elected lane of a converged warp: the whole warp runs the
+// Tensor-core products, kind::f16 (bf16 in, fp32 accumulate):
+//   umma_ss_elect: D[tmem] (+)= A[smem desc] * B[smem desc]^T;
+//   umma_ts_elect: D[tmem] (+)= A[tmem] * B[smem desc];
+//   umma_commit_elect: arrive (once) on an mbarrier when all previously issued
+//   tcgen05 ops of this thread complete.
+// Each is issued by one elected lane of a converged warp: the whole warp runs the
 // loop around them (its operands stay warp-uniform, so the compiler keeps them
 // in uniform registers) and elect.sync picks the lane that issues, inside the
 // same asm statement.
@@ -344,6 +291,8 @@ __device__ __forceinline__ void umma_commit_elect(uint32_t bar) {
       : "memory");
 }
 
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100 version 1.
+//   addr: byte address in shared memory; lbo/sbo: byte offsets (multiples of 16).
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((addr & 0x3FFFF) >> 4);
@@ -440,19 +389,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
       "r"(r[15])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
-      "%29, %30, %31, %32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-      "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
 
